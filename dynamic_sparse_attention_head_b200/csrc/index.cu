@@ -1,0 +1,643 @@
+// Index-side kernels: token layout, grid stride/phase search, materialisation of the
+// per-class row lists / gathered-key lists / line bitmaps, and the executed-tile builder.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "kernels.h"
+#include "msa_internal.h"
+
+namespace msa {
+
+namespace {
+
+template <typename T>
+__host__ __device__ __forceinline__ T* at(const DevPlan& dp, int64_t off) {
+  return reinterpret_cast<T*>(dp.ws + off);
+}
+__device__ __forceinline__ const ClassStatic& cls(const DevPlan& dp, int c) {
+  return at<const ClassStatic>(dp, dp.lay.classes)[c];
+}
+__device__ __forceinline__ const HeadStatic& head(const DevPlan& dp, int h) {
+  return at<const HeadStatic>(dp, dp.lay.heads)[h];
+}
+__device__ __forceinline__ ClassDyn& dyn(const DevPlan& dp, int c) { return at<ClassDyn>(dp, dp.lay.class_dyn)[c]; }
+
+__device__ __forceinline__ void flag_bounds(const DevPlan& dp) {
+  atomicOr(at<uint32_t>(dp, dp.lay.header), DEV_ERR_BOUNDS);
+}
+
+// ---------------------------------------------------------------------------------------
+// token layout: modality, within-modality rank, modality-grouped order (text, then video)
+// ---------------------------------------------------------------------------------------
+__global__ void layout_kernel(DevPlan dp, int64_t n_text) {
+  const int32_t* seg = at<const int32_t>(dp, dp.lay.segs);
+  uint8_t* mod = at<uint8_t>(dp, dp.lay.modality);
+  int32_t* rank = at<int32_t>(dp, dp.lay.rank);
+  int32_t* perm = at<int32_t>(dp, dp.lay.perm2d);
+  // segment s starts a run; rank base = tokens of the same modality in earlier segments
+  for (int s = blockIdx.x; s < dp.n_segs; s += gridDim.x) {
+    const int32_t st = seg[3 * s], len = seg[3 * s + 1], m = seg[3 * s + 2];
+    __shared__ int32_t base_sh;
+    if (threadIdx.x == 0) {
+      int32_t b = 0;
+      for (int q = 0; q < s; ++q)
+        if (seg[3 * q + 2] == m) b += seg[3 * q + 1];
+      base_sh = b;
+    }
+    __syncthreads();
+    const int32_t base = base_sh;
+    const int64_t region = (m == MSA_TEXT) ? 0 : n_text;
+    for (int32_t i = threadIdx.x; i < len; i += blockDim.x) {
+      const int32_t t = st + i;
+      mod[t] = (uint8_t)m;
+      rank[t] = base + i;
+      perm[region + base + i] = t;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// per-class dynamic state of classes whose rows are known at plan time
+// ---------------------------------------------------------------------------------------
+__global__ void dyn_init_kernel(DevPlan dp) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= dp.n_classes) return;
+  const ClassStatic& cs = cls(dp, c);
+  ClassDyn& d = dyn(dp, cs.dyn);
+  d.nrows = cs.rows_static < 0 ? 0 : cs.rows_static;
+  d.qrow0 = cs.qrow0_static;
+  d.x_len = 0;
+  d.n_slash = 0;
+}
+
+// ---------------------------------------------------------------------------------------
+// vertical-slash style classes (VSLASH, QBOUND, BOUND2D): gathered list, slash and
+// exclusion bitmaps.  One CTA per class.
+// ---------------------------------------------------------------------------------------
+__global__ void mat_lists_kernel(DevPlan dp) {
+  const int c = blockIdx.x;
+  const ClassStatic& cs = cls(dp, c);
+  if (!(cs.kind == MSA_VSLASH || cs.kind == MSA_QBOUND || cs.kind == MSA_BOUND2D)) return;
+  const HeadStatic& hs = head(dp, cs.head);
+  const int32_t* counts = at<const int32_t>(dp, hs.counts_off);
+  const int a = (cs.kind == MSA_VSLASH) ? 0 : cs.modality;
+  const int nwords = (int)((dp.L + 31) >> 5);
+  uint32_t* sbits = at<uint32_t>(dp, cs.slash_bits_off);
+  uint32_t* ebits = at<uint32_t>(dp, cs.excl_bits_off);
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) {
+    sbits[w] = 0u;
+    ebits[w] = 0u;
+  }
+  __syncthreads();
+  // slash lines
+  const int32_t ns = hs.raws_cap[a] > 0 ? counts[4 + a] : 0;
+  const int32_t* sl = at<const int32_t>(dp, hs.raws_off[a]);
+  for (int i = threadIdx.x; i < ns; i += blockDim.x) {
+    const int32_t o = sl[i];
+    if (o < 0 || o >= dp.L) { flag_bounds(dp); continue; }
+    atomicOr(&sbits[o >> 5], 1u << (o & 31));
+  }
+  // gathered keys: VSLASH [0][0]; QBOUND [a][0]; BOUND2D merge of [a][0] and [a][1]
+  int32_t* xp = at<int32_t>(dp, cs.x_pos_off);
+  const int32_t* ra = at<const int32_t>(dp, hs.rawv_off[a][0]);
+  const int32_t na = hs.rawv_cap[a][0] > 0 ? counts[a * 2] : 0;
+  const int32_t* rb = at<const int32_t>(dp, hs.rawv_off[a][1]);
+  const int32_t nb_ = (cs.kind == MSA_BOUND2D && hs.rawv_cap[a][1] > 0) ? counts[a * 2 + 1] : 0;
+  const int32_t nx = na + nb_;
+  if (nx > cs.x_cap) {
+    if (threadIdx.x == 0) flag_bounds(dp);
+    return;
+  }
+  const int32_t* rank = at<const int32_t>(dp, dp.lay.rank);
+  for (int i = threadIdx.x; i < na; i += blockDim.x) {
+    const int32_t v = ra[i];
+    int lo = 0, hi = nb_;  // elements of b strictly below v
+    while (lo < hi) {
+      int m = (lo + hi) >> 1;
+      if (rb[m] < v) lo = m + 1;
+      else hi = m;
+    }
+    xp[i + lo] = v;
+    if (cs.kind != MSA_BOUND2D || a == 0) {
+      const int32_t e = (cs.kind == MSA_BOUND2D) ? rank[v] : v;  // own-modality keys leave the identity region
+      atomicOr(&ebits[e >> 5], 1u << (e & 31));
+    }
+  }
+  for (int i = threadIdx.x; i < nb_; i += blockDim.x) {
+    const int32_t v = rb[i];
+    int lo = 0, hi = na;  // elements of a not above v
+    while (lo < hi) {
+      int m = (lo + hi) >> 1;
+      if (ra[m] <= v) lo = m + 1;
+      else hi = m;
+    }
+    xp[i + lo] = v;
+    if (a == 1) {
+      const int32_t e = rank[v];
+      atomicOr(&ebits[e >> 5], 1u << (e & 31));
+    }
+  }
+  for (int i = nx + threadIdx.x; i < cs.x_cap; i += blockDim.x) xp[i] = POS_PAD;
+  if (threadIdx.x == 0) {
+    ClassDyn& d = dyn(dp, cs.dyn);
+    d.x_len = nx;
+    d.n_slash = ns;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Grid stride / phase search (MMInference Algorithm 1, "key machinery"): the column sums v
+// of the last 64 video queries are averaged over the video keys of each (stride, phase);
+// the stride with the highest best-phase mean wins (ties: the smaller stride), then its
+// n_p best phases are kept (ties: the smaller phase).  One CTA per grid head.
+// ---------------------------------------------------------------------------------------
+__global__ void grid_detect_kernel(DevPlan dp) {
+  const int h = blockIdx.x;
+  const HeadStatic& hs = head(dp, h);
+  if (hs.kind != MSA_GRID) return;
+  __shared__ float sc_best[4096];
+  __shared__ float sc_cur[4096];
+  __shared__ float red_v[32];
+  __shared__ int red_i[32];
+  __shared__ int best_s_sh;
+  __shared__ float best_val_sh;
+  const RowSet* rs = nullptr;
+  for (int r = 0; r < dp.n_rowsets; ++r) {
+    const RowSet& x = at<const RowSet>(dp, dp.lay.rowsets)[r];
+    if (x.head == h) rs = &x;
+  }
+  const bool have_v = rs && rs->n_rows > 0;
+  const float* v = have_v ? at<const float>(dp, rs->v_off) : nullptr;
+  const int32_t* seg = at<const int32_t>(dp, dp.lay.segs);
+  if (threadIdx.x == 0) {
+    best_s_sh = -1;
+    best_val_sh = 0.f;
+  }
+  __syncthreads();
+  for (int ci = 0; ci < hs.grid_n_cand; ++ci) {
+    const int s = hs.grid_cand[ci];
+    float my_best = -INFINITY;
+    for (int p = threadIdx.x; p < s; p += blockDim.x) {
+      float sum = 0.f;
+      int cnt = 0;
+      for (int g = 0; g < dp.n_segs; ++g) {
+        if (seg[3 * g + 2] != MSA_VIDEO) continue;
+        const int st = seg[3 * g], len = seg[3 * g + 1];
+        for (int t = p; t < len; t += s) {
+          if (have_v) sum += v[st + t];
+          ++cnt;
+        }
+      }
+      const float mean = cnt > 0 ? sum / (float)cnt : 0.f;
+      sc_cur[p] = mean;
+      my_best = fmaxf(my_best, mean);
+    }
+    // block max of the best-phase means
+    for (int o = 16; o; o >>= 1) {
+      float ov = __shfl_xor_sync(0xFFFFFFFFu, my_best, o);
+      my_best = fmaxf(my_best, ov);
+    }
+    if ((threadIdx.x & 31) == 0) red_v[threadIdx.x >> 5] = my_best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float m = -INFINITY;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red_v[w]);
+      if (best_s_sh < 0 || m > best_val_sh) {
+        best_s_sh = ci;
+        best_val_sh = m;
+      }
+    }
+    __syncthreads();
+    if (best_s_sh == ci)
+      for (int p = threadIdx.x; p < s; p += blockDim.x) sc_best[p] = sc_cur[p];
+    __syncthreads();
+  }
+  const int ci = best_s_sh;
+  const int s = hs.grid_cand[ci];
+  const int np = hs.grid_np[ci];
+  int32_t* phases = at<int32_t>(dp, hs.phases_off);
+  // n_p rounds of (max score, smallest phase) selection
+  for (int k = 0; k < np; ++k) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int p = threadIdx.x; p < s; p += blockDim.x) {
+      const float x = sc_best[p];
+      if (x > bv || (x == bv && p < bi)) {
+        bv = x;
+        bi = p;
+      }
+    }
+    for (int o = 16; o; o >>= 1) {
+      float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+      int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((threadIdx.x & 31) == 0) {
+      red_v[threadIdx.x >> 5] = bv;
+      red_i[threadIdx.x >> 5] = bi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float b = -INFINITY;
+      int i = 0x7fffffff;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w)
+        if (red_v[w] > b || (red_v[w] == b && red_i[w] < i)) {
+          b = red_v[w];
+          i = red_i[w];
+        }
+      phases[k] = i;
+      sc_best[i] = -INFINITY;  // taken
+      // a phase scoring -inf can only be a taken one; keep the order of the rest
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    // sort the phases ascending (n_p is small)
+    for (int i = 1; i < np; ++i) {
+      int x = phases[i], j = i - 1;
+      while (j >= 0 && phases[j] > x) {
+        phases[j + 1] = phases[j];
+        --j;
+      }
+      phases[j + 1] = x;
+    }
+    int32_t* counts = at<int32_t>(dp, hs.counts_off);
+    counts[6] = s;
+    counts[7] = np;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// grid classes: marks, row lists of both classes, gathered grid keys, exclusion bitmap.
+// One CTA (1024 threads) per grid head; each thread owns a contiguous run of positions
+// whose length is a multiple of 32 so bitmap words are written without atomics.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ int block_excl_scan(int x, int* sh, int* total) {
+  // 1024 threads; sh holds 32 ints
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int v = x;
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += y;
+  }
+  if (lane == 31) sh[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    int s = sh[lane];
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      if (lane >= o) s += y;
+    }
+    sh[lane] = s;  // inclusive over warps
+  }
+  __syncthreads();
+  const int before_warp = w ? sh[w - 1] : 0;
+  *total = sh[31];
+  __syncthreads();
+  return before_warp + v - x;
+}
+
+__global__ void __launch_bounds__(1024) grid_mat_kernel(DevPlan dp) {
+  const int h = blockIdx.x;
+  const HeadStatic& hs = head(dp, h);
+  if (hs.kind != MSA_GRID) return;
+  __shared__ uint32_t pset[128];  // phase bitmap, strides <= 4096
+  __shared__ int scan_sh[32];
+  const int32_t* counts = at<const int32_t>(dp, hs.counts_off);
+  const int s = counts[6], np = counts[7];
+  const int32_t* phases = at<const int32_t>(dp, hs.phases_off);
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) pset[i] = 0u;
+  __syncthreads();
+  if (threadIdx.x < np) {
+    const int ph = phases[threadIdx.x];
+    if (ph >= 0 && ph < 4096) atomicOr(&pset[ph >> 5], 1u << (ph & 31));
+  }
+  __syncthreads();
+  const ClassStatic& c0 = cls(dp, hs.class0);
+  const ClassStatic& c1 = cls(dp, hs.class0 + 1);
+  const int64_t L = dp.L;
+  const int64_t per = ((L + blockDim.x - 1) / blockDim.x + 31) / 32 * 32;
+  const int64_t t0 = min((int64_t)threadIdx.x * per, L), t1 = min(t0 + per, L);
+  const uint8_t* mod = at<const uint8_t>(dp, dp.lay.modality);
+  const int32_t* seg = at<const int32_t>(dp, dp.lay.segs);
+  uint8_t* gm = at<uint8_t>(dp, hs.gmark_off);
+  // pass 1: marks and counts
+  int g_cnt = 0, c0_cnt = 0, c1_cnt = 0;
+  {
+    int sidx = 0;
+    // first segment overlapping t0
+    int lo = 0, hi = dp.n_segs - 1;
+    while (lo < hi) {
+      int m = (lo + hi + 1) >> 1;
+      if (seg[3 * m] <= t0) lo = m;
+      else hi = m - 1;
+    }
+    sidx = lo;
+    for (int64_t t = t0; t < t1; ++t) {
+      while (sidx + 1 < dp.n_segs && seg[3 * (sidx + 1)] <= t) ++sidx;
+      uint8_t g = 0;
+      if (mod[t] == MSA_VIDEO) {
+        const int ph = (int)((t - seg[3 * sidx]) % s);
+        g = (pset[ph >> 5] >> (ph & 31)) & 1u;
+      }
+      gm[t] = g;
+      g_cnt += g;
+      if (g || mod[t] == MSA_TEXT) ++c0_cnt;
+      else ++c1_cnt;
+    }
+  }
+  __syncthreads();
+  int g_tot, c0_tot, c1_tot;
+  const int g_off = block_excl_scan(g_cnt, scan_sh, &g_tot);
+  const int c0_off = block_excl_scan(c0_cnt, scan_sh, &c0_tot);
+  const int c1_off = block_excl_scan(c1_cnt, scan_sh, &c1_tot);
+  if (g_tot > c1.x_cap) {
+    if (threadIdx.x == 0) flag_bounds(dp);
+    return;
+  }
+  int32_t* rows0 = at<int32_t>(dp, c0.rows_off);
+  int32_t* rows1 = at<int32_t>(dp, c1.rows_off);
+  int32_t* xg = at<int32_t>(dp, c1.x_pos_off);
+  uint32_t* ex = at<uint32_t>(dp, c1.excl_bits_off);
+  {
+    int gi = g_off, i0 = c0_off, i1 = c1_off;
+    uint32_t word = 0u;
+    for (int64_t t = t0; t < t1; ++t) {
+      const uint8_t g = gm[t];
+      if (g) {
+        xg[gi++] = (int32_t)t;
+        word |= 1u << (t & 31);
+      }
+      if (g || mod[t] == MSA_TEXT) rows0[i0++] = (int32_t)t;
+      else rows1[i1++] = (int32_t)t;
+      if ((t & 31) == 31 || t == t1 - 1) {
+        ex[t >> 5] = word;
+        word = 0u;
+      }
+    }
+  }
+  for (int i = g_tot + threadIdx.x; i < c1.x_cap; i += blockDim.x) xg[i] = POS_PAD;
+  if (threadIdx.x == 0) {
+    ClassDyn& d0 = dyn(dp, c0.dyn);
+    d0.nrows = c0_tot;
+    d0.qrow0 = 0;
+    d0.x_len = 0;
+    d0.n_slash = 0;
+    ClassDyn& d1 = dyn(dp, c1.dyn);
+    d1.nrows = c1_tot;
+    d1.qrow0 = (c0_tot + TILE - 1) / TILE * TILE;
+    d1.x_len = g_tot;
+    d1.n_slash = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// block-sparse selection bitmaps: one warp per query block row
+// ---------------------------------------------------------------------------------------
+__global__ void block_bits_kernel(DevPlan dp, int c) {
+  const ClassStatic& cs = cls(dp, c);
+  const HeadStatic& hs = head(dp, cs.head);
+  const int nb = hs.blk_nb;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  uint32_t* bits = at<uint32_t>(dp, cs.blk_bits_off);
+  const int32_t* lists = at<const int32_t>(dp, hs.blk_list_off);
+  const int32_t* cnt = at<const int32_t>(dp, hs.blk_cnt_off);
+  for (int b = warp; b < nb; b += nwarps) {
+    uint32_t* row = bits + (size_t)b * cs.blk_wpr;
+    for (int w = lane; w < cs.blk_wpr; w += 32) row[w] = 0u;
+    __syncwarp();
+    const int n = cnt[b];
+    for (int i = lane; i < n; i += 32) {
+      const int kb = lists[(size_t)b * hs.blk_kmax + i];
+      if (kb < 0 || kb > b) {
+        flag_bounds(dp);
+        continue;
+      }
+      atomicOr(&row[kb >> 5], 1u << (kb & 31));
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Tile builder: one warp per 128-query work item.  Gathered-key tiles first (the keys of
+// the class's gathered list at positions <= the last query), then the identity region:
+// every condition of the class marks the 64-key units it needs (causal bound included),
+// and the marked units are covered greedily by disjoint 128-key windows starting on a
+// marked unit.  Windows may cover unneeded keys; the attention kernel's element mask
+// removes them, and disjointness guarantees no key is counted twice for a row.
+// ---------------------------------------------------------------------------------------
+constexpr int TB_WARPS = 8;
+
+__device__ __forceinline__ void mark_units(uint32_t* bm, int64_t a, int64_t b, int32_t kc_lo, int64_t hi_clip) {
+  if (a < kc_lo) a = kc_lo;
+  if (b > hi_clip) b = hi_clip;
+  if (a > b) return;
+  const int64_t ua = (a - kc_lo) >> 6, ub = (b - kc_lo) >> 6;
+  for (int64_t u = ua; u <= ub;) {
+    const int64_t w = u >> 5;
+    const int lo = (int)(u & 31);
+    const int hi = (int)(ub - (w << 5) < 31 ? ub - (w << 5) : 31);
+    const uint32_t m = (hi - lo == 31) ? 0xFFFFFFFFu : (((1u << (hi - lo + 1)) - 1u) << lo);
+    atomicOr(&bm[w], m);
+    u = (w + 1) << 5;
+  }
+}
+
+__global__ void __launch_bounds__(TB_WARPS * 32) tiles_kernel(DevPlan dp, int bm_words) {
+  extern __shared__ uint32_t tb_smem[];
+  const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* bm = tb_smem + (size_t)wl * (bm_words + 2 * TILE);
+  int32_t* run_lo = reinterpret_cast<int32_t*>(bm + bm_words);
+  int32_t* run_hi = run_lo + TILE;
+  const int wpb = blockDim.x >> 5;
+  const int gw = blockIdx.x * wpb + wl, nw = gridDim.x * wpb;
+  const WorkItem* items = at<const WorkItem>(dp, dp.lay.items);
+  int32_t* ntiles = at<int32_t>(dp, dp.lay.item_ntiles);
+  uint32_t* tiles = at<uint32_t>(dp, dp.lay.tiles);
+  for (int item = gw; item < dp.n_items; item += nw) {
+    const WorkItem wi = items[item];
+    const ClassStatic& cs = cls(dp, wi.cls);
+    const ClassDyn cd = dyn(dp, cs.dyn);
+    const int nrows = cd.nrows;
+    const int row0 = wi.slot * TILE;
+    if (row0 >= nrows) {
+      if (lane == 0) ntiles[item] = 0;
+      continue;
+    }
+    const int nval = min(TILE, nrows - row0);
+    const int32_t* rl = at<const int32_t>(dp, cs.rows_off);
+    const bool perm = (cs.flags & CF_PERMUTED) != 0;
+    const bool rank = (cs.flags & CF_RANK) != 0;
+    auto pos_of = [&](int r) -> int32_t { return perm ? rl[r] : r; };
+    auto coord_of = [&](int r) -> int32_t { return rank ? r : pos_of(r); };
+    const int32_t qpos_max = pos_of(row0 + nval - 1);
+    const int32_t qc_min = coord_of(row0), qc_max = coord_of(row0 + nval - 1);
+    uint32_t* out = tiles + cs.tile_base + (int64_t)wi.slot * cs.tile_cap;
+    int nt = 0;
+    // ---- gathered keys
+    if (cs.flags & CF_X) {
+      const int32_t* xp = at<const int32_t>(dp, cs.x_pos_off);
+      int lo = 0, hi = cd.x_len;
+      while (lo < hi) {
+        int m = (lo + hi) >> 1;
+        if (xp[m] <= qpos_max) lo = m + 1;
+        else hi = m;
+      }
+      const int ntx = (lo + TILE - 1) / TILE;
+      for (int i = lane; i < ntx; i += 32) out[i] = ((uint32_t)SRC_X << 28) | (uint32_t)(cs.x_row0 + i * TILE);
+      nt = ntx;
+    }
+    // ---- identity region
+    const int64_t hi_clip = ((int64_t)qc_max < (int64_t)cs.kc_hi - 1) ? (int64_t)qc_max : (int64_t)cs.kc_hi - 1;
+    const int64_t umax = hi_clip >= cs.kc_lo ? ((hi_clip - cs.kc_lo) >> 6) : -1;
+    const int wmax = (int)((umax + 32) >> 5);  // words in use
+    if (wmax > bm_words) {
+      if (lane == 0) {
+        flag_bounds(dp);
+        ntiles[item] = 0;
+      }
+      continue;
+    }
+    for (int w = lane; w < wmax; w += 32) bm[w] = 0u;
+    // runs of consecutive coordinates among the tile's rows
+    int nruns = 0;
+    {
+      int ne = 0;
+      for (int base = 0; base < nval; base += 32) {
+        const int r = base + lane;
+        bool start = false, end = false;
+        int32_t c = 0;
+        if (r < nval) {
+          c = coord_of(row0 + r);
+          start = (r == 0) || (coord_of(row0 + r - 1) != c - 1);
+          end = (r == nval - 1) || (coord_of(row0 + r + 1) != c + 1);
+        }
+        const uint32_t bs = __ballot_sync(0xFFFFFFFFu, start), be = __ballot_sync(0xFFFFFFFFu, end);
+        const uint32_t lt = (1u << lane) - 1u;
+        if (start) run_lo[nruns + __popc(bs & lt)] = c;
+        if (end) run_hi[ne + __popc(be & lt)] = c;
+        nruns += __popc(bs);
+        ne += __popc(be);
+      }
+      __syncwarp();
+    }
+    const int32_t kc_lo = cs.kc_lo;
+    if (umax >= 0) {
+      if (cs.flags & CF_DENSE) {
+        if (lane == 0) mark_units(bm, kc_lo, hi_clip, kc_lo, hi_clip);
+      } else {
+        if ((cs.flags & CF_SINK) && lane == 0) mark_units(bm, kc_lo, (int64_t)cs.sink - 1, kc_lo, hi_clip);
+        if (cs.flags & CF_BAND)
+          for (int i = lane; i < nruns; i += 32)
+            mark_units(bm, (int64_t)run_lo[i] - cs.band + 1, run_hi[i], kc_lo, hi_clip);
+        if (cs.flags & CF_SLASH) {
+          const int32_t* sl = at<const int32_t>(dp, cs.slash_list_off);
+          for (int i = lane; i < cd.n_slash; i += 32) {
+            const int64_t o = sl[i];
+            for (int r = 0; r < nruns; ++r) mark_units(bm, run_lo[r] - o, run_hi[r] - o, kc_lo, hi_clip);
+          }
+        }
+        if (cs.flags & CF_BLOCK) {
+          const HeadStatic& hs = head(dp, cs.head);
+          const int32_t* lists = at<const int32_t>(dp, hs.blk_list_off);
+          const int32_t* cnt = at<const int32_t>(dp, hs.blk_cnt_off);
+          for (int qb = qc_min >> 6; qb <= (qc_max >> 6); ++qb) {
+            const int n = cnt[qb];
+            for (int i = lane; i < n; i += 32) {
+              const int64_t kb = lists[(size_t)qb * hs.blk_kmax + i];
+              mark_units(bm, kb * BLK, kb * BLK + BLK - 1, kc_lo, hi_clip);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    // ---- greedy cover of the marked units by disjoint 2-unit windows (lane 0)
+    if (lane == 0) {
+      int carry = 0;
+      for (int w = 0; w < wmax; ++w) {
+        uint32_t x = bm[w];
+        if (carry) x &= ~1u;
+        carry = 0;
+        while (x) {
+          const int b = __ffs(x) - 1;
+          const int64_t u = ((int64_t)w << 5) + b;
+          if (nt < cs.tile_cap) out[nt] = ((uint32_t)cs.k_src << 28) | (uint32_t)(cs.krow_lo + u * UNIT);
+          ++nt;
+          if (b == 31) {
+            carry = 1;
+            x = 0;
+          } else {
+            x &= ~(3u << b);
+          }
+        }
+      }
+      if (nt > cs.tile_cap) {
+        flag_bounds(dp);
+        nt = cs.tile_cap;
+      }
+      ntiles[item] = nt;
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+cudaError_t launch_layout(const DevPlan& dp, cudaStream_t st) {
+  layout_kernel<<<std::min(dp.n_segs, 4096), 256, 0, st>>>(dp, dp.n_text);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grid_detect(const DevPlan& dp, cudaStream_t st) {
+  grid_detect_kernel<<<dp.Hq, 256, 0, st>>>(dp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_materialize(const DevPlan& dp, cudaStream_t st) {
+  dyn_init_kernel<<<(dp.n_classes + 127) / 128, 128, 0, st>>>(dp);
+  mat_lists_kernel<<<dp.n_classes, 512, 0, st>>>(dp);
+  grid_mat_kernel<<<dp.Hq, 1024, 0, st>>>(dp);
+  for (int c = 0; c < dp.n_classes; ++c)
+    if (dp.class_kind[c] == MSA_BLOCK) block_bits_kernel<<<std::max(1, std::min(dp.nb / 8, 1024)), 256, 0, st>>>(dp, c);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tiles(const DevPlan& dp, cudaStream_t st) {
+  const int bm_words = dp.tb_words;
+  const size_t per_warp = (size_t)(bm_words + 2 * TILE) * 4;
+  int warps = TB_WARPS;
+  while (warps > 1 && per_warp * warps > 200 * 1024) --warps;
+  const size_t smem = per_warp * warps;
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  static size_t configured = 0;
+  if (smem > 48 * 1024 && smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  const int blocks = std::max(1, std::min((dp.n_items + warps - 1) / warps, sm_count() * 8));
+  tiles_kernel<<<blocks, warps * 32, smem, st>>>(dp, bm_words);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

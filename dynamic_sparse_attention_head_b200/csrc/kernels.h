@@ -1,0 +1,51 @@
+// Host launchers of the libmsa kernels (one translation unit each).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "msa_internal.h"
+
+namespace msa {
+
+struct DevPlan {
+  uint8_t* ws;
+  Layout lay;
+  int64_t L;
+  int32_t Hq, Hkv, LP;
+  int32_t n_classes, n_heads, n_rowsets, n_jobs, n_items, n_segs;
+  int32_t x_rows;      // rows per gathered K/V slice
+  int32_t n_qslices, n_xslices;
+  int32_t has2d, has_block;
+  int32_t nb;          // L / 64
+  int64_t n_text;      // text tokens (they lead the modality-grouped order)
+  int32_t tb_words;    // unit-bitmap words per tile-builder warp
+  int32_t max_chunks;  // most key chunks of any row set
+  float scale;
+  const int32_t* class_kind;  // host copy: kind of each class
+};
+
+int sm_count();
+
+// layout of modalities / ranks / modality-grouped order from the segment table
+cudaError_t launch_layout(const DevPlan& dp, cudaStream_t st);
+// last-64-query sweeps (two passes) and top-k jobs
+cudaError_t launch_lastq(const DevPlan& dp, const void* Q, const void* K, const msa_strides& s, cudaStream_t st);
+cudaError_t launch_topk_jobs(const DevPlan& dp, cudaStream_t st);
+// block-sparse pooled estimation
+cudaError_t launch_block_estimate(const DevPlan& dp, const void* Q, const void* K, const msa_strides& s,
+                                  cudaStream_t st);
+// grid stride / phase search
+cudaError_t launch_grid_detect(const DevPlan& dp, cudaStream_t st);
+// raw index sets -> row classes, gathered lists, bitmaps, then the tile lists
+cudaError_t launch_materialize(const DevPlan& dp, cudaStream_t st);
+cudaError_t launch_tiles(const DevPlan& dp, cudaStream_t st);
+// gathers
+cudaError_t launch_permute(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
+                           cudaStream_t st);
+cudaError_t launch_unpermute(const DevPlan& dp, void* O, const msa_strides& s, cudaStream_t st);
+// attention
+cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
+                             float* lse, cudaStream_t st);
+
+}  // namespace msa

@@ -1,0 +1,213 @@
+/*
+ * msa.h - modality-aware permutation sparse attention for long-context prefill
+ * on NVIDIA B200 (sm_100a).  C ABI of libmsa.so.
+ *
+ * The method (MMInference, ICML 2025, building on MInference 1.0, NeurIPS 2024):
+ * every attention head is assigned a sparse pattern offline; online, for each
+ * prefill, a sparse index is estimated per head from the last 64 queries (or
+ * from 64-token mean-pooled blocks), Q/K/V are permuted so the selected entries
+ * become contiguous, block-sparse causal attention runs over only those blocks,
+ * and the output is permuted back.  The four steps are the four calls
+ *   msa_estimate -> msa_permute -> msa_sparse_prefill -> msa_unpermute.
+ *
+ * Conventions shared by every call
+ *  - Tensors are bf16, d = 128 contiguous elements per row.  Q and O are
+ *    [Hq, L, 128], K and V are [Hkv, L, 128], addressed through msa_strides
+ *    (element strides between heads and between rows), so [L, H, 128] works
+ *    as well.  Base pointers must be 16-byte aligned and strides multiples of
+ *    8 elements.  Query head h reads key/value head h / (Hq / Hkv).
+ *  - Causality is always j <= i in ORIGINAL token positions.
+ *  - All device pointers are owned by the caller; the library never allocates
+ *    or frees device memory.  Scratch lives in one caller-provided workspace of
+ *    msa_workspace_bytes() bytes, 256-byte aligned, which carries the estimated
+ *    indices and permuted tensors from one call to the next: pass the same
+ *    workspace to the four calls of one prefill and do not reuse it for another
+ *    prefill until the last call has completed on the stream.
+ *  - Calls are asynchronous and stream-ordered on the cudaStream_t passed as
+ *    `stream` (NULL = legacy default stream); only msa_read_indices,
+ *    msa_read_tiles and msa_device_status synchronise.
+ *  - Argument errors are returned before any launch.  Conditions found on the
+ *    device (a bounded wait that expired, an index outside its buffer) are
+ *    recorded in the workspace and reported by msa_device_status; kernels never
+ *    trap.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,   /* null pointer, unknown kind, negative budget, ... */
+  MSA_ERR_SHAPE = 2,         /* d != 128, L % 64 != 0, Hq % Hkv != 0, segments not tiling [0, L) */
+  MSA_ERR_ALIGN = 3,         /* pointer not 16-byte (workspace: 256-byte) aligned, stride not a multiple of 8 */
+  MSA_ERR_WORKSPACE = 4,     /* workspace smaller than msa_workspace_bytes() */
+  MSA_ERR_UNSUPPORTED = 5,   /* a valid problem outside this build's limits (see msa_status_string) */
+  MSA_ERR_CUDA = 6,          /* a CUDA runtime/driver call failed */
+  MSA_ERR_TIMEOUT = 7,       /* device: a bounded wait expired (reported by msa_device_status) */
+  MSA_ERR_DEVICE_BOUNDS = 8, /* device: an index fell outside its buffer (reported by msa_device_status) */
+  MSA_ERR_STATE = 9          /* calls out of order for this workspace */
+} msa_status;
+
+/* modality of a token */
+enum { MSA_TEXT = 0, MSA_VIDEO = 1 };
+
+/* Sparse pattern of one attention head (MInference 1.0, "Approach"; MMInference, "key machinery").
+ *  DENSE   : causal attention, no sparsity.
+ *  ASHAPE  : attention sinks + local window: j < sink or i - j < local (static, no estimation).
+ *  VSLASH  : vertical lines V (keys) and slash lines S (offsets i - j), top k_v / k_s of the
+ *            last-64-query attention reduced per key / per offset.
+ *  BLOCK   : 64x64 blocks; per query block the top-k key blocks of the mean-pooled logits.
+ *  GRID    : video grid (MMInference Algorithm 1): stride s and phases P searched online from
+ *            the last 64 video queries; queries and keys on the (s, P) lines attend / are attended
+ *            densely, text queries attend densely, plus a local band of `local` (default 64).
+ *  QBOUND  : Q-boundary (Algorithm 2): vertical-slash per query modality.
+ *  BOUND2D : 2D-boundary (Algorithm 3): per (query modality, key modality) pair; intra-modality
+ *            pairs are vertical-slash in within-modality ranks, cross pairs vertical only. */
+typedef enum {
+  MSA_DENSE = 0,
+  MSA_ASHAPE = 1,
+  MSA_VSLASH = 2,
+  MSA_BLOCK = 3,
+  MSA_GRID = 4,
+  MSA_QBOUND = 5,
+  MSA_BOUND2D = 6
+} msa_kind;
+
+#define MSA_MAX_STRIDES 8
+
+typedef struct {
+  int32_t kind;        /* msa_kind */
+  int32_t sink;        /* ASHAPE: sink tokens */
+  int32_t local;       /* ASHAPE: local window; GRID: local band (0 = 64) */
+  int32_t k_v;         /* VSLASH/QBOUND: vertical lines; BOUND2D: scaled per key modality, max(1, round(k_v n_b / L)) */
+  int32_t k_s;         /* VSLASH/QBOUND: slash lines;    BOUND2D: max(1, round(k_s n_a / L)) per query modality */
+  int32_t topk_blocks; /* BLOCK: key blocks per query block (> 0), else block_budget is used */
+  double block_budget; /* BLOCK: keep ceil(block_budget * (b + 1)) blocks in query block b */
+  int32_t n_strides;   /* GRID: candidate strides (1..MSA_MAX_STRIDES) */
+  int32_t strides[MSA_MAX_STRIDES];
+  int32_t n_phases;    /* GRID: phases kept (> 0), else max(1, floor(grid_budget * s / 2)) */
+  int32_t _pad;
+  double grid_budget;
+} msa_head_cfg;
+
+typedef struct {
+  int64_t start, len; /* token range [start, start + len) */
+  int32_t modality;   /* MSA_TEXT or MSA_VIDEO */
+  int32_t _pad;
+} msa_segment;
+
+typedef struct {
+  int64_t L;                   /* sequence length, a multiple of 64 */
+  int32_t Hq, Hkv, d;          /* d must be 128; Hq a multiple of Hkv */
+  float scale;                 /* softmax scale, e.g. 1/sqrt(128) */
+  int32_t n_segments;          /* ordered segments tiling [0, L) */
+  const msa_segment* segments; /* host pointer, copied by msa_plan_create */
+  const msa_head_cfg* heads;   /* host pointer [Hq], copied by msa_plan_create */
+} msa_problem;
+
+/* element strides of the four tensors; the 128-element d axis is contiguous */
+typedef struct {
+  int64_t q_head, q_row;
+  int64_t k_head, k_row;
+  int64_t v_head, v_row;
+  int64_t o_head, o_row;
+} msa_strides;
+
+typedef struct msa_plan msa_plan;
+
+/* Validates the problem and sizes the workspace.  Host only: no device work, no
+ * allocation on the device.  On success *out owns a host copy of every table. */
+msa_status msa_plan_create(const msa_problem* problem, msa_plan** out);
+void msa_plan_destroy(msa_plan* plan);
+
+/* Bytes of device workspace one prefill with this plan needs. */
+size_t msa_workspace_bytes(const msa_plan* plan);
+
+/* Online index estimation (MInference 1.0 "Approach": last-64-query vertical/slash sums,
+ * 64-block mean pooling; MMInference "key machinery": grid stride/phase search, per-modality
+ * estimation from the 64 latest queries of every modality), followed by the
+ * per-head row classes, gathered-key lists, line bitmaps and executed-tile lists.
+ * Reads Q and K (device), writes only the workspace. */
+msa_status msa_estimate(msa_plan* plan, const void* Q, const void* K, const msa_strides* strides, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* Host-provided index sets instead of msa_estimate (indices reused across prefills, or fixed
+ * ones).  One msa_head_indices per query head; fields a head's kind does not use are ignored.
+ * Lists are host pointers, sorted ascending, copied before the call returns. */
+typedef struct {
+  int32_t stride;          /* GRID: chosen stride */
+  int32_t n_phases;        /* GRID: phases (< stride) */
+  const int32_t* phases;
+  int32_t n_v[2][2];       /* vertical lines, token positions: VSLASH [0][0]; QBOUND [a][0] for query
+                              modality a over all keys; BOUND2D [a][b] keys of modality b */
+  const int32_t* v[2][2];
+  int32_t n_s[2];          /* slash lines (offsets): VSLASH [0]; QBOUND [a]; BOUND2D [a] in ranks */
+  const int32_t* s[2];
+  const int32_t* blk_ptr;  /* BLOCK: CSR over query blocks, blk_ptr[L/64 + 1] */
+  const int32_t* blk_idx;  /* BLOCK: selected key blocks (each row ascending, c <= b) */
+} msa_head_indices;
+
+msa_status msa_set_indices(msa_plan* plan, const msa_head_indices* heads, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Permutation (MMInference "core discovery": row-wise grouping of same-modality queries,
+ * column-wise gathering of selected keys, 2D modality-pair grouping).  Gathers permuted Q
+ * rows, gathered K/V lines and modality-grouped K/V into the workspace. */
+msa_status msa_permute(msa_plan* plan, const void* Q, const void* K, const void* V, const msa_strides* strides,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Block-sparse causal flash attention over the executed tiles (MMInference "key machinery":
+ * kernels that load only the permuted blocks and keep the tensor-core compute dense;
+ * "Grid-Shape Flash Attention", Algorithm 5).  Writes the permuted output into the workspace
+ * and, if lse != NULL, the natural-log softmax normaliser per query, lse[h * L + i] (fp32,
+ * -inf for a query with no allowed key; such a query's output row is 0). */
+msa_status msa_sparse_prefill(msa_plan* plan, const void* Q, const void* K, const void* V,
+                              const msa_strides* strides, void* ws, size_t ws_bytes, float* lse, void* stream);
+
+/* Scatters the permuted output back to original token order into O (bf16, device). */
+msa_status msa_unpermute(msa_plan* plan, const void* ws, size_t ws_bytes, void* O, const msa_strides* strides,
+                         void* stream);
+
+/* ---- inspection (synchronising) ---- */
+
+/* Copies head `head`'s raw index sets to the host as a flat int32 record:
+ *   kind, stride, n_phases, phases[n_phases],
+ *   for a in {0,1}, b in {0,1}: n_v[a][b], v[a][b][...],
+ *   for a in {0,1}: n_s[a], s[a][...],
+ *   nb, blk_ptr[nb + 1], blk_idx[blk_ptr[nb]]          (nb = 0 unless BLOCK)
+ * `*len` is the capacity of `out` in int32 on entry and the record length on return
+ * (MSA_ERR_INVALID_ARG with the needed length if too small). */
+msa_status msa_read_indices(const msa_plan* plan, const void* ws, int32_t head, int32_t* out, int64_t* len,
+                            void* stream);
+
+/* Executed-tile statistics of the last msa_estimate / msa_set_indices in this workspace:
+ * tiles[0] = executed 128x128 tiles, tiles[1] = work items (128-query tiles) with work.
+ * Executed block FLOPs = 4 * 128 * 128 * 128 * tiles[0]. */
+msa_status msa_tile_stats(const msa_plan* plan, const void* ws, int64_t tiles[2], void* stream);
+
+/* Dumps the work list of head `head` for tests: for each of its 128-query work items the
+ * query positions covered (-1 for padding) and, for every executed tile, its key source
+ * (0 = keys in original order, 1 = modality-grouped keys, 2 = gathered keys) and the original
+ * positions of its 128 keys (-1 where a column holds no key, or a key the tile's mask leaves
+ * to a gathered tile).  Flat int32 record:
+ *   n_items, then per item: class, n_rows, rows[128], n_tiles, n_tiles x (src, keys[128]).
+ * `*len` as for msa_read_indices. */
+msa_status msa_read_tiles(const msa_plan* plan, const void* ws, int32_t head, int32_t* out, int64_t* len,
+                          void* stream);
+
+/* Synchronises `stream` and returns the first device-side error recorded in `ws` (MSA_OK if
+ * none) and clears it. */
+msa_status msa_device_status(const msa_plan* plan, void* ws, void* stream);
+
+const char* msa_status_string(msa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_H_ */

@@ -37,10 +37,9 @@ static inline float logit(const uint16_t* q, const uint16_t* k, int d, float sca
 }
 
 /*
- * Last-query attention sums (MInference 1.0, "Approach": the vertical and slash
- * lines are estimated from the attention of the last 64 queries; MMInference,
- * "core discovery": the sparse index is estimated from the last 64 queries of
- * each modality segment).
+ * Last-query attention sums (MInference 1.0, section "Approach": vertical and
+ * slash lines come from the attention rows of the final 64 queries; MMInference,
+ * "core discovery": video-aware heads take those 64 rows per modality).
  *
  * For each estimation row r (original position rows[r]) the causal softmax
  * A[r, j] = exp(x_rj - m_r) / Z_r over all keys j <= rows[r] is formed, and

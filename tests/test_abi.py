@@ -1,0 +1,63 @@
+"""The C-ABI library builds, loads and exports every symbol include/msa.h declares; host-only
+argument validation of msa_plan_create (no GPU needed: plan creation does no device work)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    return sorted(set(re.findall(r"^(?:msa_status|void|size_t|const char\*)\s+(msa_\w+)\(", src, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    from dynamic_sparse_attention_head_b200 import build
+    lib = ctypes.CDLL(build.build())
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"libmsa.so does not export {n}"
+
+
+def test_binding_names_match_header():
+    import dynamic_sparse_attention_head_b200 as msa
+    assert sorted(msa.EXPORTS) == _declared()
+
+
+def test_plan_validation_is_host_only():
+    import dynamic_sparse_attention_head_b200 as msa
+    from workload import TEXT, Head, Problem, llama3_8b_text
+
+    p = msa.Plan(llama3_8b_text(L=4096))
+    assert p.workspace_bytes > 0
+
+    class Bad:
+        pass
+
+    def prob(**kw):
+        b = Bad()
+        b.L, b.Hq, b.Hkv, b.d, b.scale = 1024, 2, 1, 128, 0.088
+        b.segments = [(0, 1024, TEXT)]
+        b.heads = [Head("dense")] * 2
+        for k, v in kw.items():
+            setattr(b, k, v)
+        return b
+
+    for kw, code in ((dict(L=1000, segments=[(0, 1000, TEXT)]), 2), (dict(d=64), 2), (dict(Hkv=3), 2),
+                     (dict(segments=[(0, 512, TEXT)]), 2), (dict(heads=[Head("vslash")] * 2), 1),
+                     (dict(heads=[Head("grid")] * 2), 1), (dict(scale=0.0), 1)):
+        with pytest.raises(msa.MsaError) as e:
+            msa.Plan(prob(**kw))
+        assert e.value.code == code, kw
+
+
+def test_workspace_grows_with_length():
+    import dynamic_sparse_attention_head_b200 as msa
+    from workload import llama3_8b_text
+    a = msa.Plan(llama3_8b_text(L=4096)).workspace_bytes
+    b = msa.Plan(llama3_8b_text(L=8192)).workspace_bytes
+    assert b > a
