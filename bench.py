@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the modality-aware permutation sparse prefill path on B200.
+
+One step = one attention layer through the whole hot path on one batch of synthetic input:
+msa_estimate -> msa_permute -> msa_sparse_prefill -> msa_unpermute.
+
+metric: sparse-prefill attention ms/layer + effective TFLOP/s (executed 128x128 block FLOPs,
+4 * 128^3 per tile) at 128K and 1M tokens.  `value` is effective TFLOP/s of the whole step,
+summed over ranks (each rank runs its own layer: weak scaling, no collective on the data path).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workload  # noqa: E402
+
+METRIC = "sparse-prefill attention ms/layer + effective TFLOP/s at 128K and 1M tokens"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def workloads():
+    W = {
+        "qwen2-7b-video-128k": workload.qwen2_7b_video_128k,
+        "longvila-1m": workload.longvila_1m,
+        "llama3-8b-text-32k": lambda: workload.llama3_8b_text(L=32768),
+        "grid-1head-4k": lambda: workload.grid_single_head(),
+        "qwen2-7b-video-64f": workload.qwen2_7b_video_literal,
+    }
+    for L in workload.SWEEP_LENGTHS:
+        W[f"sweep-dense-L{L}"] = (lambda L=L: workload.sweep_layer(L, None))
+        for b in workload.SWEEP_BUDGETS:
+            W[f"sweep-b{int(round(b * 100))}-L{L}"] = (lambda L=L, b=b: workload.sweep_layer(L, b))
+    return W
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kind_summary(p):
+    from collections import Counter
+    c = Counter(h.kind for h in p.heads)
+    return " / ".join(f"{n} {k}" for k, n in c.items())
+
+
+def dense_causal_flops(p):
+    return 2 * p.d * p.L * (p.L + 1) * p.Hq
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = uuid
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                sm.append(float(f[2]))
+                mx.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 f[6:10]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle on a bounded sample (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------------------
+def oracle_sample(p, Q, K, V, rows_per_head=32, seed=0):
+    """Times the oracle on one head of each kind: its full index estimation plus masked
+    attention for `rows_per_head` uniformly sampled query rows, the attention time scaled by
+    L / rows (attention time is proportional to rows on a uniform sample).  Returns per-kind
+    seconds for one head and the sampled heads."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    heads = {}
+    for h, hd in enumerate(p.heads):
+        heads.setdefault(hd.kind, h)
+    per_kind = {}
+    for kind, h in heads.items():
+        t0 = time.perf_counter()
+        idx = oracle.estimate_head(p, h, Q, K)
+        t1 = time.perf_counter()
+        rows = np.sort(rng.choice(p.L, size=min(rows_per_head, p.L), replace=False))
+        oracle.attention_head(p, h, Q, K, V, idx, rows)
+        t2 = time.perf_counter()
+        per_kind[kind] = {"head": h, "est_s": t1 - t0, "attn_s": (t2 - t1) * p.L / len(rows), "idx": idx}
+    return per_kind
+
+
+def oracle_layer_seconds(p, per_kind):
+    from collections import Counter
+    n = Counter(h.kind for h in p.heads)
+    return sum(n[k] * (v["est_s"] + v["attn_s"]) for k, v in per_kind.items())
+
+
+def cores():
+    return len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------------------------------
+def make_host_inputs(p, seed):
+    Q, K, V = workload.make_inputs(p, seed=seed)
+    return Q, K, V
+
+
+def attn_source_hash():
+    h = hashlib.sha256()
+    for f in ("attn.cu", "ptx.cuh", "msa_internal.h"):
+        with open(os.path.join(ROOT, "dynamic_sparse_attention_head_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary, if the
+    kernel source still matches the one the counters were taken on."""
+    path = os.path.join(ROOT, "profiles", "attn_dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(workload_name)
+    if not ent or ent.get("attn_source_hash") != attn_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import dynamic_sparse_attention_head_b200 as msa
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    p = workloads()[args.workload]()
+    Qh, Kh, Vh = make_host_inputs(p, seed=rank)
+
+    def dev_copy(x):
+        return torch.from_numpy(x).view(torch.bfloat16).to(dev)
+
+    q, k, v = dev_copy(Qh), dev_copy(Kh), dev_copy(Vh)
+    o = torch.empty_like(q)
+    plan = msa.Plan(p)
+    ws = plan.alloc_workspace()
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        if events is not None:
+            events[0].record(stream)
+        plan.estimate(q, k, ws)
+        if events is not None:
+            events[1].record(stream)
+        plan.permute(q, k, v, ws)
+        if events is not None:
+            events[2].record(stream)
+        plan.sparse_prefill(q, k, v, ws)
+        if events is not None:
+            events[3].record(stream)
+        plan.unpermute(ws, o)
+        if events is not None:
+            events[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = plan.device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    tiles, items = plan.tile_stats(ws)
+    exec_flops = msa.executed_flops(tiles)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(local_rank).uuid)
+    except Exception:
+        uuid = None
+    n0 = msa.kernel_launches()
+    with ClockSampler(uuid) as clk:
+        start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        end.record(stream)
+        torch.cuda.synchronize()
+    launches = msa.kernel_launches() - n0
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # ms
+    # max over ranks of the timed region; sum of executed FLOPs over ranks
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        f = torch.tensor([float(exec_flops)], device=dev, dtype=torch.float64)
+        dist.all_reduce(f, op=dist.ReduceOp.SUM)
+        job_flops = float(f.item())
+    else:
+        job_flops = float(exec_flops)
+    ms_step = total_ms / args.steps
+    value = job_flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers: H2D inputs, path, D2H output
+    e2e = None
+    if not args.no_e2e:
+        qp = torch.from_numpy(Qh).view(torch.bfloat16).pin_memory()
+        kp = torch.from_numpy(Kh).view(torch.bfloat16).pin_memory()
+        vp = torch.from_numpy(Vh).view(torch.bfloat16).pin_memory()
+        op = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            step()
+            op.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        bi = (Qh.nbytes + Kh.nbytes + Vh.nbytes)
+        bo = int(np.prod(o.shape)) * 2
+        e2e = {"value": job_flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps}
+
+    pk, pk_src = peaks()
+    attn_ms = float(stage[:, 2].mean())
+    achieved = exec_flops / (attn_ms * 1e-3) / 1e12
+    peak_sus = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    traffic = recorded_traffic(args.workload)
+    roofline = {"kernel": "msa_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": peak_sus,
+                "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
+                "peak_source": f"{pk_src} bf16_tflops_sustained (kernel inside a long step)",
+                "frac_of_burst_peak": achieved / peak_burst,
+                "flops_per_launch": exec_flops, "ms_per_launch": attn_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_kind = oracle_sample(p, Qh, Kh, Vh, rows_per_head=args.cpu_rows)
+        layer_s = oracle_layer_seconds(p, per_kind)
+        cpu = {"value": exec_flops / layer_s / 1e12, "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
+               "ms_per_layer": layer_s * 1e3,
+               "sample": (f"oracle on one head of each kind ({', '.join(per_kind)}): full index estimation + "
+                          f"masked attention of {args.cpu_rows} uniformly sampled rows scaled to L rows; "
+                          f"layer time = sum over heads of their kind's time; value = this layer's executed "
+                          f"block FLOPs / that time")}
+
+    if rank == 0:
+        sm = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "ms_per_layer": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
+                       "heads": kind_summary(p), "parallelism": f"independent layer per rank x{world}",
+                       "l2": "inputs larger than L2 (no flush)" if (Qh.nbytes > 126e6) else "inputs smaller than L2",
+                       "seed": "rank"},
+            "stages_ms": {"estimate": float(stage[:, 0].mean()), "permute": float(stage[:, 1].mean()),
+                          "attention": attn_ms, "unpermute": float(stage[:, 3].mean())},
+            "executed_tiles": tiles, "work_items": items, "executed_flops": exec_flops,
+            "dense_causal_flops": dense_causal_flops(p),
+            "dense_flops_avoided": dense_causal_flops(p) - exec_flops,
+            "attn_tflops": achieved,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": sm,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: bounded samples of the same workload on host cores."""
+    if rank != 0:
+        return
+    p = workloads()[args.workload]()
+    Qh, Kh, Vh = make_host_inputs(p, seed=0)
+    flops = None
+    # executed block FLOPs of the sampled heads' oracle indices, counted by the tile builder
+    # (untimed, only to express the oracle's time in the metric's unit)
+    per_kind = None
+    times = []
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        per_kind = oracle_sample(p, Qh, Kh, Vh, rows_per_head=args.cpu_rows, seed=s)
+        t = oracle_layer_seconds(p, per_kind)
+        if s >= args.warmup:
+            times.append(t)
+        _ = time.perf_counter() - t0
+    flops = executed_flops_for(p, per_kind)
+    layer_s = float(np.mean(times))
+    value = flops / layer_s / 1e12 if flops else None
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": layer_s * 1e3, "ms_per_layer": layer_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
+                       "heads": kind_summary(p)},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
+                             "sample": (f"per step: oracle on one head of each kind, full estimation + "
+                                        f"{args.cpu_rows} sampled rows of masked attention scaled to L rows; "
+                                        f"layer time summed over heads by kind")},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def executed_flops_for(p, per_kind):
+    """Executed block FLOPs of the whole layer when each head uses its kind's sampled oracle
+    index set (tile builder run on the GPU, untimed).  None without a GPU."""
+    try:
+        import torch
+        if not torch.cuda.is_available():
+            return None
+        import dynamic_sparse_attention_head_b200 as msa
+    except Exception:
+        return None
+    idx = [per_kind[h.kind]["idx"] for h in p.heads]
+    if any(h.kind == "block" for h in p.heads):
+        pass
+    plan = msa.Plan(p)
+    ws = plan.alloc_workspace()
+    plan.set_indices(idx, ws)
+    tiles, _ = plan.tile_stats(ws)
+    return msa.executed_flops(tiles)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="qwen2-7b-video-128k", choices=sorted(workloads()))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=32)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -74,6 +74,7 @@ def _load():
         "msa_tile_stats": ([_P, _P, _P, _P], _I32),
         "msa_device_status": ([_P, _P, _P], _I32),
         "msa_status_string": ([_I32], ctypes.c_char_p),
+        "msa_kernel_launches": ([], ctypes.c_uint64),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -85,7 +86,12 @@ def _load():
 _lib = _load()
 EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_estimate", "msa_set_indices",
            "msa_permute", "msa_sparse_prefill", "msa_unpermute", "msa_read_indices", "msa_read_tiles",
-           "msa_tile_stats", "msa_device_status", "msa_status_string")
+           "msa_tile_stats", "msa_device_status", "msa_status_string", "msa_kernel_launches")
+
+
+def kernel_launches() -> int:
+    """Kernels launched by libmsa since it was loaded."""
+    return int(_lib.msa_kernel_launches())
 
 
 def _check(fn: str, code: int):

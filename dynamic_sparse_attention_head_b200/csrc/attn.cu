@@ -587,6 +587,7 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
     configured = true;
   }
   const int grid = std::max(1, std::min(dp.n_items, sm_count()));
+  count_launches(1);
   msa_attn_kernel<<<grid, ATT_THREADS, smem, st>>>(mq, mqp, mk, mv, mk2, mv2, mxk, mxv, p);
   return cudaGetLastError();
 }

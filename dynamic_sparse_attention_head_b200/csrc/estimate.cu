@@ -545,12 +545,14 @@ __global__ void __launch_bounds__(BT_THREADS) block_topk_kernel(DevPlan dp) {
 
 // ---------------------------------------------------------------------------------------
 cudaError_t launch_group_k(const DevPlan& dp, const void* K, const msa_strides& s, cudaStream_t st) {
+  count_launches(1);
   group_rows_kernel<<<sm_count() * 8, 256, 0, st>>>(dp, static_cast<const __nv_bfloat16*>(K), s.k_head, s.k_row,
                                                    at<__nv_bfloat16>(dp, dp.lay.k2d));
   return cudaGetLastError();
 }
 
 cudaError_t launch_group_v(const DevPlan& dp, const void* V, const msa_strides& s, cudaStream_t st) {
+  count_launches(1);
   group_rows_kernel<<<sm_count() * 8, 256, 0, st>>>(dp, static_cast<const __nv_bfloat16*>(V), s.v_head, s.v_row,
                                                    at<__nv_bfloat16>(dp, dp.lay.v2d));
   return cudaGetLastError();
@@ -569,6 +571,7 @@ cudaError_t launch_lastq(const DevPlan& dp, const void* Q, const void* K, const 
   }
   const dim3 grid(dp.max_chunks, dp.n_rowsets);
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
+  count_launches(3);
   lastq_pass1<<<grid, LQ_THREADS, smem1, st>>>(dp, q, s.q_head, s.q_row, K, s.k_head, s.k_row);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   lastq_combine<<<dp.n_rowsets, LASTQ, 0, st>>>(dp);
@@ -578,6 +581,7 @@ cudaError_t launch_lastq(const DevPlan& dp, const void* Q, const void* K, const 
 }
 
 cudaError_t launch_topk_jobs(const DevPlan& dp, cudaStream_t st) {
+  count_launches(1);
   topk_jobs_kernel<<<dp.n_jobs, TK_THREADS, 0, st>>>(dp);
   return cudaGetLastError();
 }
@@ -585,6 +589,7 @@ cudaError_t launch_topk_jobs(const DevPlan& dp, cudaStream_t st) {
 cudaError_t launch_block_estimate(const DevPlan& dp, const void* Q, const void* K, const msa_strides& s,
                                   cudaStream_t st) {
   const int gx = std::min(dp.nb, 1024);
+  count_launches(3);
   pool_kernel<<<dim3(gx, dp.Hkv), D, 0, st>>>(dp, static_cast<const __nv_bfloat16*>(K), s.k_head, s.k_row, dp.Hkv,
                                               0);
   pool_kernel<<<dim3(gx, dp.Hq), D, 0, st>>>(dp, static_cast<const __nv_bfloat16*>(Q), s.q_head, s.q_row, dp.Hq, 1);

@@ -604,21 +604,27 @@ int sm_count() {
 }
 
 cudaError_t launch_layout(const DevPlan& dp, cudaStream_t st) {
+  count_launches(1);
   layout_kernel<<<std::min(dp.n_segs, 4096), 256, 0, st>>>(dp, dp.n_text);
   return cudaGetLastError();
 }
 
 cudaError_t launch_grid_detect(const DevPlan& dp, cudaStream_t st) {
+  count_launches(1);
   grid_detect_kernel<<<dp.Hq, 256, 0, st>>>(dp);
   return cudaGetLastError();
 }
 
 cudaError_t launch_materialize(const DevPlan& dp, cudaStream_t st) {
+  count_launches(3);
   dyn_init_kernel<<<(dp.n_classes + 127) / 128, 128, 0, st>>>(dp);
   mat_lists_kernel<<<dp.n_classes, 512, 0, st>>>(dp);
   grid_mat_kernel<<<dp.Hq, 1024, 0, st>>>(dp);
   for (int c = 0; c < dp.n_classes; ++c)
-    if (dp.class_kind[c] == MSA_BLOCK) block_bits_kernel<<<std::max(1, std::min(dp.nb / 8, 1024)), 256, 0, st>>>(dp, c);
+    if (dp.class_kind[c] == MSA_BLOCK) {
+      count_launches(1);
+      block_bits_kernel<<<std::max(1, std::min(dp.nb / 8, 1024)), 256, 0, st>>>(dp, c);
+    }
   return cudaGetLastError();
 }
 
@@ -636,6 +642,7 @@ cudaError_t launch_tiles(const DevPlan& dp, cudaStream_t st) {
     configured = smem;
   }
   const int blocks = std::max(1, std::min((dp.n_items + warps - 1) / warps, sm_count() * 8));
+  count_launches(1);
   tiles_kernel<<<blocks, warps * 32, smem, st>>>(dp, bm_words);
   return cudaGetLastError();
 }

@@ -26,6 +26,8 @@ struct DevPlan {
 };
 
 int sm_count();
+// bumps the library-wide kernel launch counter by n
+void count_launches(int n);
 
 // layout of modalities / ranks / modality-grouped order from the segment table
 cudaError_t launch_layout(const DevPlan& dp, cudaStream_t st);

@@ -121,15 +121,24 @@ cudaError_t launch_permute(const DevPlan& dp, const void* Q, const void* K, cons
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
   const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K);
   const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(V);
-  if (dp.n_qslices > 0) permute_q_kernel<<<dim3(bx * 2, dp.Hq), 256, 0, st>>>(dp, q, s.q_head, s.q_row);
-  if (dp.n_xslices > 0)
+  if (dp.n_qslices > 0) {
+    count_launches(1);
+    permute_q_kernel<<<dim3(bx * 2, dp.Hq), 256, 0, st>>>(dp, q, s.q_head, s.q_row);
+  }
+  if (dp.n_xslices > 0) {
+    count_launches(1);
     gather_x_kernel<<<dim3(bx, dp.Hq), 256, 0, st>>>(dp, k, s.k_head, s.k_row, v, s.v_head, s.v_row);
-  if (dp.has2d) group_kv_kernel<<<sm_count() * 8, 256, 0, st>>>(dp, k, s.k_head, s.k_row, v, s.v_head, s.v_row);
+  }
+  if (dp.has2d) {
+    count_launches(1);
+    group_kv_kernel<<<sm_count() * 8, 256, 0, st>>>(dp, k, s.k_head, s.k_row, v, s.v_head, s.v_row);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpermute(const DevPlan& dp, void* O, const msa_strides& s, cudaStream_t st) {
   const int bx = std::max(1, sm_count() * 8 / std::max(1, dp.Hq));
+  count_launches(1);
   unpermute_kernel<<<dim3(bx, dp.Hq), 256, 0, st>>>(dp, static_cast<__nv_bfloat16*>(O), s.o_head, s.o_row);
   return cudaGetLastError();
 }

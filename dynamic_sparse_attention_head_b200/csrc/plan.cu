@@ -15,6 +15,13 @@
 
 using namespace msa;
 
+#include <atomic>
+
+namespace msa {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace msa
+
 struct msa_plan {
   int64_t L = 0;
   int32_t Hq = 0, Hkv = 0;
@@ -110,6 +117,8 @@ std::vector<int32_t> last_rows(const msa_plan& P, int a, int n = LASTQ) {
 }  // namespace
 
 extern "C" {
+
+uint64_t msa_kernel_launches(void) { return msa::g_launches.load(std::memory_order_relaxed); }
 
 const char* msa_status_string(msa_status s) {
   switch (s) {

@@ -207,6 +207,10 @@ msa_status msa_device_status(const msa_plan* plan, void* ws, void* stream);
 
 const char* msa_status_string(msa_status status);
 
+/* Number of CUDA kernels this library has launched since it was loaded (all plans, all
+ * threads); lets a caller count the kernels of one call by differencing. */
+uint64_t msa_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

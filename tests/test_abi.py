@@ -11,7 +11,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def _declared():
     src = open(os.path.join(ROOT, "include", "msa.h")).read()
-    return sorted(set(re.findall(r"^(?:msa_status|void|size_t|const char\*)\s+(msa_\w+)\(", src, re.M)))
+    return sorted(set(re.findall(r"^(?:msa_status|void|size_t|uint64_t|const char\*)\s+(msa_\w+)\(", src, re.M)))
 
 
 def test_library_exports_every_declared_symbol():
