@@ -37,7 +37,7 @@ struct AttnParams {
   float* lse;              // [Hq][L] or null
 };
 
-constexpr int ATT_THREADS = 256;
+constexpr int ATT_THREADS = 384;  // 0 TMA, 1 MMA, 2-3 spare, 4-11 softmax (two warpgroups)
 constexpr int KV_STAGES = 2;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // one 128x128 bf16 tile
 constexpr uint32_t ATOM_BYTES = 128 * 128;      // one [128 rows][64 cols] 128B-swizzled atom
@@ -52,6 +52,8 @@ struct __align__(1024) AttnSmem {
   uint64_t v_full[KV_STAGES], v_empty[KV_STAGES];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, pv_done, o_free, drain;
+  float xmax[2][2][128];  // [tile parity][warpgroup][row] partial row max
+  float xsum[2][128];     // [warpgroup][row] partial row sum
   uint32_t tmem_base;
   int abort;
 };
@@ -93,29 +95,7 @@ __device__ __forceinline__ bool load_item(const AttnParams& p, int item, ItemInf
   return it.ntiles >= 0;
 }
 
-__device__ __forceinline__ void prefix_mask(uint32_t (&m)[4], int n) {
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    int k = n - 32 * w;
-    m[w] = k >= 32 ? 0xFFFFFFFFu : (k <= 0 ? 0u : ((1u << k) - 1u));
-  }
-}
-
-// 128 bits of a global bitmap starting at (possibly negative) bit `base`.
-__device__ __forceinline__ void bits128(const uint32_t* bm, int nwords, int base, uint32_t (&o)[4]) {
-  const int w0 = base >> 5;  // floor division
-  const int sh = base & 31;
-  uint32_t x[5];
-#pragma unroll
-  for (int i = 0; i < 5; ++i) {
-    int w = w0 + i;
-    x[i] = (w >= 0 && w < nwords) ? __ldg(bm + w) : 0u;
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(x[i], x[i + 1], sh);
-}
-
-// Allowed-key mask of one query row against the 128 keys of a tile (bit c = key column c).
+// Per-row state of the element mask.
 struct RowCtx {
   int valid, qpos, qcoord;
   int flags, sink, band, kc_lo, kc_hi, krow_lo, x_row0, nwords, blk_wpr;
@@ -125,54 +105,76 @@ struct RowCtx {
   const int32_t* xpos;
 };
 
-__device__ __forceinline__ void tile_mask(const RowCtx& rc, int src, int krow, uint32_t (&m)[4]) {
+// 64 bits of a global bitmap starting at (possibly negative) bit `base`.
+__device__ __forceinline__ void bits64(const uint32_t* bm, int nwords, int base, uint32_t (&o)[2]) {
+  const int w0 = base >> 5;
+  const int sh = base & 31;
+  uint32_t x[3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    int w = w0 + i;
+    x[i] = (w >= 0 && w < nwords) ? __ldg(bm + w) : 0u;
+  }
+  o[0] = __funnelshift_r(x[0], x[1], sh);
+  o[1] = __funnelshift_r(x[1], x[2], sh);
+}
+
+__device__ __forceinline__ void prefix_mask2(uint32_t (&m)[2], int n) {
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    int k = n - 32 * w;
+    m[w] = k >= 32 ? 0xFFFFFFFFu : (k <= 0 ? 0u : ((1u << k) - 1u));
+  }
+}
+
+// Allowed-key mask of one query row against key columns [64 half, 64 half + 64) of a tile.
+__device__ __forceinline__ void tile_mask_half(const RowCtx& rc, int src, int krow, int half, uint32_t (&m)[2]) {
   if (!rc.valid) {
-    m[0] = m[1] = m[2] = m[3] = 0u;
+    m[0] = m[1] = 0u;
     return;
   }
   if (src == SRC_X) {
     // gathered keys are sorted by position: the allowed ones are a prefix
-    const int32_t* kp = rc.xpos + (krow - rc.x_row0);
-    int lo = 0, hi = 128;
+    const int32_t* kp = rc.xpos + (krow - rc.x_row0) + 64 * half;
+    int lo = 0, hi = 64;
     while (lo < hi) {
       int mid = (lo + hi) >> 1;
       if (__ldg(kp + mid) <= rc.qpos) lo = mid + 1;
       else hi = mid;
     }
-    prefix_mask(m, lo);
+    prefix_mask2(m, lo);
     return;
   }
-  const int kc0 = rc.kc_lo + (krow - rc.krow_lo);  // coordinate of column 0
-  int n = min(rc.qcoord - kc0 + 1, rc.kc_hi - kc0);
-  prefix_mask(m, n);                               // causal and inside the region
+  const int kc0 = rc.kc_lo + (krow - rc.krow_lo) + 64 * half;  // coordinate of this half's column 0
+  prefix_mask2(m, min(rc.qcoord - kc0 + 1, rc.kc_hi - kc0));  // causal and inside the region
   if (!(rc.flags & CF_DENSE)) {
-    uint32_t any[4] = {0u, 0u, 0u, 0u};
+    uint32_t any[2] = {0u, 0u};
     if (rc.flags & CF_SINK) {
-      uint32_t t[4];
-      prefix_mask(t, rc.sink - kc0);
-#pragma unroll
-      for (int w = 0; w < 4; ++w) any[w] |= t[w];
+      uint32_t t[2];
+      prefix_mask2(t, rc.sink - kc0);
+      any[0] |= t[0];
+      any[1] |= t[1];
     }
     if (rc.flags & CF_BAND) {
-      uint32_t t[4];
-      prefix_mask(t, rc.qcoord - rc.band + 1 - kc0);  // columns below qcoord - band + 1 are outside
-#pragma unroll
-      for (int w = 0; w < 4; ++w) any[w] |= ~t[w];
+      uint32_t t[2];
+      prefix_mask2(t, rc.qcoord - rc.band + 1 - kc0);  // columns below qcoord - band + 1 are outside
+      any[0] |= ~t[0];
+      any[1] |= ~t[1];
     }
     if (rc.flags & CF_SLASH) {
-      // column c has offset qcoord - kc0 - c; gather offsets [base, base + 128) and reverse
-      uint32_t b[4];
-      bits128(rc.slash, rc.nwords, rc.qcoord - kc0 - 127, b);
-#pragma unroll
-      for (int w = 0; w < 4; ++w) any[w] |= __brev(b[3 - w]);
+      // column c has offset qcoord - kc0 - c; gather offsets [base, base + 64) and reverse
+      uint32_t b[2];
+      bits64(rc.slash, rc.nwords, rc.qcoord - kc0 - 63, b);
+      any[0] |= __brev(b[1]);
+      any[1] |= __brev(b[0]);
     }
     if (rc.flags & CF_BLOCK) {
       const uint32_t* row = rc.blk + (size_t)(rc.qcoord >> 6) * rc.blk_wpr;
+      const int nbk = (rc.kc_hi + 63) >> 6;  // key blocks of the row
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < 2; ++w) {
         const int c0 = kc0 + 32 * w;
         const int b0 = c0 >> 6, b1 = (c0 + 31) >> 6;
-        const int nbk = (rc.kc_hi + 63) >> 6;  // key blocks of the row
         const uint32_t s0 = b0 < nbk ? (__ldg(row + (b0 >> 5)) >> (b0 & 31)) & 1u : 0u;
         const uint32_t s1 = b1 < nbk ? (__ldg(row + (b1 >> 5)) >> (b1 & 31)) & 1u : 0u;
         const int split = 64 - (c0 & 63);  // columns of this word inside block b0
@@ -180,15 +182,19 @@ __device__ __forceinline__ void tile_mask(const RowCtx& rc, int src, int krow, u
         any[w] |= (s0 ? low : 0u) | (s1 ? ~low : 0u);
       }
     }
-#pragma unroll
-    for (int w = 0; w < 4; ++w) m[w] &= any[w];
+    m[0] &= any[0];
+    m[1] &= any[1];
   }
   if (rc.flags & CF_EXCL) {
-    uint32_t e[4];
-    bits128(rc.excl, rc.nwords, kc0, e);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) m[w] &= ~e[w];
+    uint32_t e[2];
+    bits64(rc.excl, rc.nwords, kc0, e);
+    m[0] &= ~e[0];
+    m[1] &= ~e[1];
   }
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void issue_kv(const CUtensorMap* tk, const CUtensorMap* tv, const CUtensorMap* tk2,
@@ -239,11 +245,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 128);
+      mbar_init(&sm.s_free[b], 256);
     }
-    mbar_init(&sm.p_full, 128);
+    mbar_init(&sm.p_full, 256);
     mbar_init(&sm.pv_done, 1);
-    mbar_init(&sm.o_free, 128);
+    mbar_init(&sm.o_free, 256);
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
@@ -355,11 +361,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ softmax / epilogue
-    const int t = threadIdx.x - 128;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+    // Two warpgroups share each tile: warpgroup g owns key columns [64g, 64g + 64) of S and
+    // output columns [64g, 64g + 64) of O; thread t owns query row t (TMEM lane t).
+    const int g = (warp - 4) >> 2;
+    const int t = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(p.ws + p.lay.op));
     const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
-    uint32_t s_count = 0, pv_waits = 0, items_done = 0;
+    uint32_t s_count = 0, pv_waits = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       ItemInfo it;
@@ -384,32 +393,35 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       rc.excl = reinterpret_cast<const uint32_t*>(p.ws + cs.excl_bits_off);
       rc.blk = reinterpret_cast<const uint32_t*>(p.ws + cs.blk_bits_off);
       rc.xpos = reinterpret_cast<const int32_t*>(p.ws + cs.x_pos_off);
-      const size_t orow = ((size_t)it.head * p.LP + it.qrow0 + r) * D;
+      const size_t orow = ((size_t)it.head * p.LP + it.qrow0 + r) * D + 64 * g;
 
       if (it.ntiles == 0) {
         if (rc.valid) {
-          uint4 z = make_uint4(0, 0, 0, 0);
           uint4* dst = reinterpret_cast<uint4*>(op + orow);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) dst[i] = z;
-          if (p.lse) p.lse[(size_t)it.head * p.L + rc.qpos] = -INFINITY;
+          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+          if (p.lse && g == 0) p.lse[(size_t)it.head * p.L + rc.qpos] = -INFINITY;
         }
         continue;
       }
 
       float m_used = -INFINITY, l = 0.f;
+      uint32_t mk[2];
+      uint32_t tile = __ldg(tiles + it.tile0);
+      tile_mask_half(rc, (int)(tile >> 28), (int)(tile & 0x0FFFFFFFu), g, mk);
       for (int tt = 0; tt < it.ntiles; ++tt) {
-        const uint32_t tile = __ldg(tiles + it.tile0 + tt);
-        uint32_t mk[4];
-        tile_mask(rc, (int)(tile >> 28), (int)(tile & 0x0FFFFFFFu), mk);
+        // mask of the next tile is computed while this one is processed
+        uint32_t mk_next[2] = {0u, 0u};
+        const bool has_next = tt + 1 < it.ntiles;
+        uint32_t tile_next = has_next ? __ldg(tiles + it.tile0 + tt + 1) : 0u;
 
         const uint32_t sb = s_count & 1, su = s_count >> 1;
         if (!mbar_wait(&sm.s_full[sb], su & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        float s[128];
-        const uint32_t scol = lane_base + (sb ? TM_S1 : TM_S0);
+        float s[64];
+        const uint32_t scol = lane_base + (sb ? TM_S1 : TM_S0) + 64 * g;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t rr[32];
           tmem_ld32(scol + 32 * c, rr);
           tmem_wait_ld();
@@ -419,28 +431,35 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         tc_fence_before();
         mbar_arrive(&sm.s_free[sb]);
         ++s_count;
+        if (has_next) tile_mask_half(rc, (int)(tile_next >> 28), (int)(tile_next & 0x0FFFFFFFu), g, mk_next);
 
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = ((mk[c >> 5] >> (c & 31)) & 1u) ? s[c] * p.scale_log2 : -INFINITY;
+        for (int c = 0; c < 64; ++c) {
+          const float x = ((mk[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
           s[c] = x;
           mx = fmaxf(mx, x);
         }
+        // row max over both halves of the tile
+        const int par = tt & 1;
+        sm.xmax[par][g][t] = mx;
+        named_bar_sync(1, 256);
+        mx = fmaxf(mx, sm.xmax[par][g ^ 1][t]);
+        const float mxs = mx * p.scale_log2;
         float alpha = 1.f;
         bool resc = false;
-        if (mx > m_used + 8.f) {  // also true on the first finite max
-          alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - mx);
-          m_used = mx;
+        if (mxs > m_used + 8.f) {  // also true on the first finite max
+          alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - mxs);
+          m_used = mxs;
           resc = true;
         }
-        const float mbase = (m_used == -INFINITY) ? 0.f : m_used;
+        const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
         float rs = 0.f;
-        uint32_t pk[64];
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float a = ex2(s[2 * c] - mbase);
-          const float b = ex2(s[2 * c + 1] - mbase);
+        for (int c = 0; c < 32; ++c) {
+          const float a = ex2(fmaf(s[2 * c], p.scale_log2, nb));
+          const float b = ex2(fmaf(s[2 * c + 1], p.scale_log2, nb));
           rs += a + b;
           pk[c] = pack_bf16x2(a, b);
         }
@@ -454,43 +473,45 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           if (__any_sync(0xFFFFFFFFu, resc)) {
             const float f = resc ? alpha : 1.f;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
               uint32_t oo[32];
-              tmem_ld32(lane_base + TM_O + 32 * c, oo);
+              const uint32_t oc = lane_base + TM_O + 64 * g + 32 * c;
+              tmem_ld32(oc, oo);
               tmem_wait_ld();
 #pragma unroll
               for (int j = 0; j < 32; ++j) oo[j] = __float_as_uint(__uint_as_float(oo[j]) * f);
-              tmem_st32(lane_base + TM_O + 32 * c, oo);
+              tmem_st32(oc, oo);
             }
             tmem_wait_st();
           }
         }
-        // P row t, K-major 128B swizzle: atom (keys 64a..64a+63), 16-byte chunk j -> j ^ (t & 7)
-        uint8_t* prow = sm.p + t * 128;
+        // P row t, K-major 128B swizzle: atom g holds keys 64g..64g+63; chunk j -> j ^ (t & 7)
+        uint8_t* prow = sm.p + g * ATOM_BYTES + t * 128;
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int w = a * 32 + j * 4;
-            uint4 v = make_uint4(pk[w], pk[w + 1], pk[w + 2], pk[w + 3]);
-            *reinterpret_cast<uint4*>(prow + a * ATOM_BYTES + ((j ^ (t & 7)) << 4)) = v;
-          }
+        for (int j = 0; j < 8; ++j) {
+          uint4 v = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          *reinterpret_cast<uint4*>(prow + ((j ^ (t & 7)) << 4)) = v;
         }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.p_full);
+        mk[0] = mk_next[0];
+        mk[1] = mk_next[1];
       }
       if (!ok) break;
-      // epilogue: last P V, then O / l
+      // epilogue: last P V, then O / l with l summed over both halves
       if (!mbar_wait(&sm.pv_done, pv_waits & 1, abort)) { ok = false; break; }
       ++pv_waits;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint32_t ov[64];
+      sm.xsum[g][t] = l;
+      named_bar_sync(1, 256);
+      const float ltot = l + sm.xsum[g ^ 1][t];
+      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+      uint32_t ov[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t oo[32];
-        tmem_ld32(lane_base + TM_O + 32 * c, oo);
+        tmem_ld32(lane_base + TM_O + 64 * g + 32 * c, oo);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j)
@@ -498,14 +519,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&sm.o_free);
-      ++items_done;
       if (rc.valid) {
         uint4* dst = reinterpret_cast<uint4*>(op + orow);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
-        if (p.lse)
+        for (int i = 0; i < 8; ++i) dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+        if (p.lse && g == 0)
           p.lse[(size_t)it.head * p.L + rc.qpos] =
-              (l > 0.f) ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+              (ltot > 0.f) ? (m_used + __log2f(ltot)) * 0.6931471805599453f : -INFINITY;
       }
     }
   }
