@@ -7,7 +7,8 @@
 //  - warp 0 streams Q, K and V tiles with TMA (128-byte swizzle) into a 2-stage ring;
 //  - warp 1 (one elected thread) issues tcgen05.mma: S = Q K^T into one of two TMEM
 //    buffers, then O += P V with O resident in TMEM for the whole work item;
-//  - warps 4..7 own TMEM lanes 0..127 (one query row per thread): they read S with
+//  - warps 2..9 form two warpgroups, each owning TMEM lanes 0..127 (one query row per thread)
+//    and one 64-key half of every tile: they read S with
 //    tcgen05.ld, apply the element mask (causal in original positions + the head's
 //    pattern), run the online softmax in fp32 (exp2 on MUFU, lazy rescale of O when the
 //    running max grows by more than 2^8), write P as bf16 into shared memory in the
@@ -37,7 +38,7 @@ struct AttnParams {
   float* lse;              // [Hq][L] or null
 };
 
-constexpr int ATT_THREADS = 384;  // 0 TMA, 1 MMA, 2-3 spare, 4-11 softmax (two warpgroups)
+constexpr int ATT_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (two warpgroups)
 constexpr int KV_STAGES = 2;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // one 128x128 bf16 tile
 constexpr uint32_t ATOM_BYTES = 128 * 128;      // one [128 rows][64 cols] 128B-swizzled atom
@@ -51,15 +52,15 @@ struct __align__(1024) AttnSmem {
   uint64_t k_full[KV_STAGES], k_empty[KV_STAGES];
   uint64_t v_full[KV_STAGES], v_empty[KV_STAGES];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, o_free, drain;
-  float xmax[2][2][128];  // [tile parity][warpgroup][row] partial row max
-  float xsum[2][128];     // [warpgroup][row] partial row sum
+  uint64_t p_full[2], pv_done[2], o_free, drain;
+  float xm[2][2][128];  // [item parity][key half][row] running max of the half (log2 units)
+  float xl[2][2][128];  // [item parity][key half][row] running sum of the half
   uint32_t tmem_base;
   int abort;
 };
 
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;  // O of key half g at TM_O + 128 g
 
 __device__ __forceinline__ const ClassStatic& class_of(const AttnParams& p, int c) {
   return reinterpret_cast<const ClassStatic*>(p.ws + p.lay.classes)[c];
@@ -105,20 +106,6 @@ struct RowCtx {
   const int32_t* xpos;
 };
 
-// 64 bits of a global bitmap starting at (possibly negative) bit `base`.
-__device__ __forceinline__ void bits64(const uint32_t* bm, int nwords, int base, uint32_t (&o)[2]) {
-  const int w0 = base >> 5;
-  const int sh = base & 31;
-  uint32_t x[3];
-#pragma unroll
-  for (int i = 0; i < 3; ++i) {
-    int w = w0 + i;
-    x[i] = (w >= 0 && w < nwords) ? __ldg(bm + w) : 0u;
-  }
-  o[0] = __funnelshift_r(x[0], x[1], sh);
-  o[1] = __funnelshift_r(x[1], x[2], sh);
-}
-
 __device__ __forceinline__ void prefix_mask2(uint32_t (&m)[2], int n) {
 #pragma unroll
   for (int w = 0; w < 2; ++w) {
@@ -127,15 +114,50 @@ __device__ __forceinline__ void prefix_mask2(uint32_t (&m)[2], int n) {
   }
 }
 
-// Allowed-key mask of one query row against key columns [64 half, 64 half + 64) of a tile.
-__device__ __forceinline__ void tile_mask_half(const RowCtx& rc, int src, int krow, int half, uint32_t (&m)[2]) {
+// Mask words of one query row against key columns [64 half, 64 half + 64) of a tile, in two
+// steps so the bitmap loads of the next tile are in flight while the current tile is
+// processed: mask_prefetch issues the loads, mask_finish combines them.
+struct MaskRaw {
+  int src, krow, kc0;
+  uint32_t sl[3], ex[3], bk0, bk1;
+};
+
+__device__ __forceinline__ uint32_t ldg_word(const uint32_t* bm, int nwords, int w) {
+  return (w >= 0 && w < nwords) ? __ldg(bm + w) : 0u;
+}
+
+__device__ __forceinline__ void mask_prefetch(const RowCtx& rc, uint32_t tile, int half, MaskRaw& r) {
+  r.src = (int)(tile >> 28);
+  r.krow = (int)(tile & 0x0FFFFFFFu);
+  r.kc0 = rc.kc_lo + (r.krow - rc.krow_lo) + 64 * half;
+  if (!rc.valid || r.src == SRC_X) return;
+  if (rc.flags & CF_SLASH) {
+    const int w0 = (rc.qcoord - r.kc0 - 63) >> 5;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) r.sl[i] = ldg_word(rc.slash, rc.nwords, w0 + i);
+  }
+  if (rc.flags & CF_EXCL) {
+    const int w0 = r.kc0 >> 5;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) r.ex[i] = ldg_word(rc.excl, rc.nwords, w0 + i);
+  }
+  if (rc.flags & CF_BLOCK) {
+    const uint32_t* row = rc.blk + (size_t)(rc.qcoord >> 6) * rc.blk_wpr;
+    const int nbk = (rc.kc_hi + 63) >> 6;
+    const int b0 = r.kc0 >> 6, b1 = b0 + 1;  // a 64-column half touches at most two blocks
+    r.bk0 = b0 < nbk ? (__ldg(row + (b0 >> 5)) >> (b0 & 31)) & 1u : 0u;
+    r.bk1 = b1 < nbk ? (__ldg(row + (b1 >> 5)) >> (b1 & 31)) & 1u : 0u;
+  }
+}
+
+__device__ __forceinline__ void mask_finish(const RowCtx& rc, const MaskRaw& r, int half, uint32_t (&m)[2]) {
   if (!rc.valid) {
     m[0] = m[1] = 0u;
     return;
   }
-  if (src == SRC_X) {
+  if (r.src == SRC_X) {
     // gathered keys are sorted by position: the allowed ones are a prefix
-    const int32_t* kp = rc.xpos + (krow - rc.x_row0) + 64 * half;
+    const int32_t* kp = rc.xpos + (r.krow - rc.x_row0) + 64 * half;
     int lo = 0, hi = 64;
     while (lo < hi) {
       int mid = (lo + hi) >> 1;
@@ -145,7 +167,7 @@ __device__ __forceinline__ void tile_mask_half(const RowCtx& rc, int src, int kr
     prefix_mask2(m, lo);
     return;
   }
-  const int kc0 = rc.kc_lo + (krow - rc.krow_lo) + 64 * half;  // coordinate of this half's column 0
+  const int kc0 = r.kc0;
   prefix_mask2(m, min(rc.qcoord - kc0 + 1, rc.kc_hi - kc0));  // causal and inside the region
   if (!(rc.flags & CF_DENSE)) {
     uint32_t any[2] = {0u, 0u};
@@ -162,34 +184,29 @@ __device__ __forceinline__ void tile_mask_half(const RowCtx& rc, int src, int kr
       any[1] |= ~t[1];
     }
     if (rc.flags & CF_SLASH) {
-      // column c has offset qcoord - kc0 - c; gather offsets [base, base + 64) and reverse
-      uint32_t b[2];
-      bits64(rc.slash, rc.nwords, rc.qcoord - kc0 - 63, b);
-      any[0] |= __brev(b[1]);
-      any[1] |= __brev(b[0]);
+      // column c has offset qcoord - kc0 - c: bits [base, base + 64) reversed
+      const int sh = (rc.qcoord - kc0 - 63) & 31;
+      const uint32_t b0 = __funnelshift_r(r.sl[0], r.sl[1], sh), b1 = __funnelshift_r(r.sl[1], r.sl[2], sh);
+      any[0] |= __brev(b1);
+      any[1] |= __brev(b0);
     }
     if (rc.flags & CF_BLOCK) {
-      const uint32_t* row = rc.blk + (size_t)(rc.qcoord >> 6) * rc.blk_wpr;
-      const int nbk = (rc.kc_hi + 63) >> 6;  // key blocks of the row
+      // columns before the next 64-boundary of the coordinate lie in block kc0 >> 6
+      const int split = 64 - (kc0 & 63);
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
-        const int c0 = kc0 + 32 * w;
-        const int b0 = c0 >> 6, b1 = (c0 + 31) >> 6;
-        const uint32_t s0 = b0 < nbk ? (__ldg(row + (b0 >> 5)) >> (b0 & 31)) & 1u : 0u;
-        const uint32_t s1 = b1 < nbk ? (__ldg(row + (b1 >> 5)) >> (b1 & 31)) & 1u : 0u;
-        const int split = 64 - (c0 & 63);  // columns of this word inside block b0
-        const uint32_t low = split >= 32 ? 0xFFFFFFFFu : ((1u << split) - 1u);
-        any[w] |= (s0 ? low : 0u) | (s1 ? ~low : 0u);
+        const int lo = split - 32 * w;  // columns of word w inside the first block
+        const uint32_t low = lo >= 32 ? 0xFFFFFFFFu : (lo <= 0 ? 0u : ((1u << lo) - 1u));
+        any[w] |= (r.bk0 ? low : 0u) | (r.bk1 ? ~low : 0u);
       }
     }
     m[0] &= any[0];
     m[1] &= any[1];
   }
   if (rc.flags & CF_EXCL) {
-    uint32_t e[2];
-    bits64(rc.excl, rc.nwords, kc0, e);
-    m[0] &= ~e[0];
-    m[1] &= ~e[1];
+    const int sh = kc0 & 31;
+    m[0] &= ~__funnelshift_r(r.ex[0], r.ex[1], sh);
+    m[1] &= ~__funnelshift_r(r.ex[1], r.ex[2], sh);
   }
 }
 
@@ -247,8 +264,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.s_free[b], 256);
     }
-    mbar_init(&sm.p_full, 256);
-    mbar_init(&sm.pv_done, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&sm.p_full[g], 128);
+      mbar_init(&sm.pv_done[g], 1);
+    }
     mbar_init(&sm.o_free, 256);
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
@@ -315,19 +334,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         ++q_uses;
         auto do_pv = [&](int t) -> bool {
           const uint32_t st = pv_count % KV_STAGES, use = pv_count / KV_STAGES;
-          if (!mbar_wait(&sm.p_full, p_uses & 1, abort)) return false;
-          ++p_uses;
           if (!mbar_wait(&sm.v_full[st], use & 1, abort)) return false;
           if (t == 0 && items_done > 0 && !mbar_wait(&sm.o_free, (items_done - 1) & 1, abort)) return false;
-          tc_fence_after();
           const uint32_t v_addr = smem_addr(sm.v[st]);
+          // O_g += P[:, 64g:64g+64] V[64g:64g+64, :] for each key half g, as soon as its P is ready
+          for (int g = 0; g < 2; ++g) {
+            if (!mbar_wait(&sm.p_full[g], p_uses & 1, abort)) return false;
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * ATOM_BYTES + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, ATOM_BYTES, 1024);
-            umma_ss(tmem + TM_O, ad, bd, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc_sw128(p_addr + g * ATOM_BYTES + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(v_addr + g * 8192 + kk * 2048, ATOM_BYTES, 1024);
+              umma_ss(tmem + TM_O + 128 * g, ad, bd, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&sm.pv_done[g]);
           }
-          umma_commit(&sm.pv_done);
+          ++p_uses;
           umma_commit(&sm.v_empty[st]);
           ++pv_count;
           return true;
@@ -359,16 +381,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       umma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, abort, 100000000ull);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------------ softmax / epilogue
-    // Two warpgroups share each tile: warpgroup g owns key columns [64g, 64g + 64) of S and
-    // output columns [64g, 64g + 64) of O; thread t owns query row t (TMEM lane t).
-    const int g = (warp - 4) >> 2;
-    const int t = (warp & 3) * 32 + lane;
+    // Two independent warpgroups: warpgroup g owns key columns [64g, 64g + 64) of every S
+    // tile with its own running max / sum and its own accumulator O_g = sum P_g V_g in TMEM;
+    // the halves are combined once per work item.  Thread t owns query row t (TMEM lane t).
+    const int g = (warp - 2) >> 2;  // warps 2-5: key half 0, warps 6-9: key half 1
+    const int t = (warp & 3) * 32 + lane;  // a warp may only touch TMEM lanes 32 (warp % 4) .. + 31
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t o_own = lane_base + TM_O + 128 * g;
     __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(p.ws + p.lay.op));
     const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
-    uint32_t s_count = 0, pv_waits = 0;
+    uint32_t s_count = 0, pv_waits = 0, items_done = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       ItemInfo it;
@@ -407,13 +431,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
       float m_used = -INFINITY, l = 0.f;
       uint32_t mk[2];
-      uint32_t tile = __ldg(tiles + it.tile0);
-      tile_mask_half(rc, (int)(tile >> 28), (int)(tile & 0x0FFFFFFFu), g, mk);
+      MaskRaw raw;
+      mask_prefetch(rc, __ldg(tiles + it.tile0), g, raw);
+      mask_finish(rc, raw, g, mk);
       for (int tt = 0; tt < it.ntiles; ++tt) {
-        // mask of the next tile is computed while this one is processed
-        uint32_t mk_next[2] = {0u, 0u};
         const bool has_next = tt + 1 < it.ntiles;
-        uint32_t tile_next = has_next ? __ldg(tiles + it.tile0 + tt + 1) : 0u;
+        if (has_next) mask_prefetch(rc, __ldg(tiles + it.tile0 + tt + 1), g, raw);
 
         const uint32_t sb = s_count & 1, su = s_count >> 1;
         if (!mbar_wait(&sm.s_full[sb], su & 1, abort)) { ok = false; break; }
@@ -431,21 +454,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         tc_fence_before();
         mbar_arrive(&sm.s_free[sb]);
         ++s_count;
-        if (has_next) tile_mask_half(rc, (int)(tile_next >> 28), (int)(tile_next & 0x0FFFFFFFu), g, mk_next);
 
-        float mx = -INFINITY;
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float x = ((mk[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
           s[c] = x;
-          mx = fmaxf(mx, x);
+          mx4[c & 3] = fmaxf(mx4[c & 3], x);
         }
-        // row max over both halves of the tile
-        const int par = tt & 1;
-        sm.xmax[par][g][t] = mx;
-        named_bar_sync(1, 256);
-        mx = fmaxf(mx, sm.xmax[par][g ^ 1][t]);
-        const float mxs = mx * p.scale_log2;
+        const float mxs = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
         float alpha = 1.f;
         bool resc = false;
         if (mxs > m_used + 8.f) {  // also true on the first finite max
@@ -453,80 +470,94 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           m_used = mxs;
           resc = true;
         }
-        const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
-        float rs = 0.f;
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float a = ex2(fmaf(s[2 * c], p.scale_log2, nb));
-          const float b = ex2(fmaf(s[2 * c + 1], p.scale_log2, nb));
-          rs += a + b;
-          pk[c] = pack_bf16x2(a, b);
-        }
-        l = l * alpha + rs;
-
-        // previous P V must be complete before P is overwritten or O rescaled
+        // the previous P_g V_g must be complete before P_g is overwritten or O_g rescaled
         if (tt > 0) {
-          if (!mbar_wait(&sm.pv_done, pv_waits & 1, abort)) { ok = false; break; }
+          if (!mbar_wait(&sm.pv_done[g], pv_waits & 1, abort)) { ok = false; break; }
           ++pv_waits;
           tc_fence_after();
           if (__any_sync(0xFFFFFFFFu, resc)) {
             const float f = resc ? alpha : 1.f;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              uint32_t oo[32];
-              const uint32_t oc = lane_base + TM_O + 64 * g + 32 * c;
-              tmem_ld32(oc, oo);
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {  // 16 columns at a time: S stays live in registers
+              uint32_t oo[16];
+              tmem_ld16(o_own + 16 * c, oo);
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) oo[j] = __float_as_uint(__uint_as_float(oo[j]) * f);
-              tmem_st32(oc, oo);
+              for (int j = 0; j < 16; ++j) oo[j] = __float_as_uint(__uint_as_float(oo[j]) * f);
+              tmem_st16(o_own + 16 * c, oo);
             }
             tmem_wait_st();
           }
         }
+        const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
         // P row t, K-major 128B swizzle: atom g holds keys 64g..64g+63; chunk j -> j ^ (t & 7)
         uint8_t* prow = sm.p + g * ATOM_BYTES + t * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint4 v = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          *reinterpret_cast<uint4*>(prow + ((j ^ (t & 7)) << 4)) = v;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float a = ex2(fmaf(s[32 * h + 2 * c], p.scale_log2, nb));
+            const float b = ex2(fmaf(s[32 * h + 2 * c + 1], p.scale_log2, nb));
+            rs4[c & 3] += a + b;
+            pk[c] = pack_bf16x2(a, b);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 v = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            *reinterpret_cast<uint4*>(prow + (((4 * h + j) ^ (t & 7)) << 4)) = v;
+          }
         }
+        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&sm.p_full);
-        mk[0] = mk_next[0];
-        mk[1] = mk_next[1];
+        mbar_arrive(&sm.p_full[g]);
+        if (has_next) mask_finish(rc, raw, g, mk);
       }
       if (!ok) break;
-      // epilogue: last P V, then O / l with l summed over both halves
-      if (!mbar_wait(&sm.pv_done, pv_waits & 1, abort)) { ok = false; break; }
+      // epilogue: both halves' last P V done, then O = (c0 O_0 + c1 O_1) / (c0 l0 + c1 l1)
+      if (!mbar_wait(&sm.pv_done[g], pv_waits & 1, abort)) { ok = false; break; }
       ++pv_waits;
-      tc_fence_after();
-      sm.xsum[g][t] = l;
+      const int ip = items_done & 1;
+      sm.xm[ip][g][t] = m_used;
+      sm.xl[ip][g][t] = l;
+      tc_fence_before();
       named_bar_sync(1, 256);
-      const float ltot = l + sm.xsum[g ^ 1][t];
+      tc_fence_after();
+      const float m0 = sm.xm[ip][0][t], m1 = sm.xm[ip][1][t];
+      const float M = fmaxf(m0, m1);
+      const float c0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M);
+      const float c1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
+      const float ltot = c0 * sm.xl[ip][0][t] + c1 * sm.xl[ip][1][t];
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-      uint32_t ov[32];
+      const float f0 = c0 * inv, f1 = c1 * inv;
+      uint4* dst = reinterpret_cast<uint4*>(op + orow);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t oo[32];
-        tmem_ld32(lane_base + TM_O + 64 * g + 32 * c, oo);
+        uint32_t oa[32], ob[32];
+        tmem_ld32(lane_base + TM_O + 64 * g + 32 * c, oa);
+        tmem_ld32(lane_base + TM_O + 128 + 64 * g + 32 * c, ob);
         tmem_wait_ld();
+        if (c == 1) {
+          tc_fence_before();
+          mbar_arrive(&sm.o_free);
+        }
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          ov[16 * c + j] = pack_bf16x2(__uint_as_float(oo[2 * j]) * inv, __uint_as_float(oo[2 * j + 1]) * inv);
-      }
-      tc_fence_before();
-      mbar_arrive(&sm.o_free);
-      if (rc.valid) {
-        uint4* dst = reinterpret_cast<uint4*>(op + orow);
+        for (int j = 0; j < 4; ++j) {
+          uint32_t w[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
-        if (p.lse && g == 0)
-          p.lse[(size_t)it.head * p.L + rc.qpos] =
-              (ltot > 0.f) ? (m_used + __log2f(ltot)) * 0.6931471805599453f : -INFINITY;
+          for (int e = 0; e < 4; ++e) {
+            const int k = 8 * j + 2 * e;
+            w[e] = pack_bf16x2(__uint_as_float(oa[k]) * f0 + __uint_as_float(ob[k]) * f1,
+                               __uint_as_float(oa[k + 1]) * f0 + __uint_as_float(ob[k + 1]) * f1);
+          }
+          if (rc.valid) dst[4 * c + j] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
       }
+      ++items_done;
+      if (rc.valid && p.lse && g == 0)
+        p.lse[(size_t)it.head * p.L + rc.qpos] = (ltot > 0.f) ? (M + __log2f(ltot)) * 0.6931471805599453f : -INFINITY;
     }
   }
 
