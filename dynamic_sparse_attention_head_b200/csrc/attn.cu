@@ -39,25 +39,28 @@ struct AttnParams {
 };
 
 constexpr int ATT_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (two warpgroups)
-constexpr int KV_STAGES = 2;
+constexpr int K_STAGES = 2;  // K tiles are loaded ahead of V tiles
+constexpr int V_STAGES = 2;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // one 128x128 bf16 tile
 constexpr uint32_t ATOM_BYTES = 128 * 128;      // one [128 rows][64 cols] 128B-swizzled atom
 
 struct __align__(1024) AttnSmem {
   uint8_t q[TILE_BYTES];
-  uint8_t k[KV_STAGES][TILE_BYTES];
-  uint8_t v[KV_STAGES][TILE_BYTES];
+  uint8_t k[K_STAGES][TILE_BYTES];
+  uint8_t v[V_STAGES][TILE_BYTES];
   uint8_t p[TILE_BYTES];
   uint64_t q_full, q_empty;
-  uint64_t k_full[KV_STAGES], k_empty[KV_STAGES];
-  uint64_t v_full[KV_STAGES], v_empty[KV_STAGES];
+  uint64_t k_full[K_STAGES], k_empty[K_STAGES];
+  uint64_t v_full[V_STAGES], v_empty[V_STAGES];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], pv_done[2], o_free, drain;
-  float xm[2][2][128];  // [item parity][key half][row] running max of the half (log2 units)
-  float xl[2][2][128];  // [item parity][key half][row] running sum of the half
+  float xm[2][128];  // [key half][row] running max of the half (log2 units)
+  float xl[2][128];  // [key half][row] running sum of the half
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(AttnSmem) <= 232448, "attention shared memory exceeds 227 KB per CTA");
 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;  // O of key half g at TM_O + 128 g
@@ -210,6 +213,12 @@ __device__ __forceinline__ void mask_finish(const RowCtx& rc, const MaskRaw& r, 
   }
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
@@ -243,8 +252,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmK2, const __grid_constant__ CUtensorMap tmV2,
                     const __grid_constant__ CUtensorMap tmXK, const __grid_constant__ CUtensorMap tmXV,
                     const AttnParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
+  if (smem_addr(smem_raw) & 1023u) {  // the 128-byte swizzled tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicOr(reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.ws + p.lay.header)), DEV_ERR_BOUNDS);
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort = &sm.abort;
@@ -254,9 +267,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     sm.abort = 0;
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
+    for (int s = 0; s < K_STAGES; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < V_STAGES; ++s) {
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
@@ -284,7 +299,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      uint32_t kv_count = 0, q_uses = 0;
+      uint32_t k_issued = 0, v_issued = 0, q_uses = 0;
       const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -300,23 +315,35 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           tma_load_3d(sm.q, &tmQ, &sm.q_full, 0, it.row0, it.head);
           tma_load_3d(sm.q + ATOM_BYTES, &tmQ, &sm.q_full, 64, it.row0, it.head);
         }
-        for (int t = 0; t < it.ntiles; ++t) {
-          const uint32_t tile = __ldg(tiles + it.tile0 + t);
-          const uint32_t st = kv_count % KV_STAGES, use = kv_count / KV_STAGES;
-          if (use > 0 && !mbar_wait(&sm.k_empty[st], (use - 1) & 1, abort)) { ok = false; break; }
-          issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, false, tile, it, sm.k[st], &sm.k_full[st]);
-          if (use > 0 && !mbar_wait(&sm.v_empty[st], (use - 1) & 1, abort)) { ok = false; break; }
-          issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, true, tile, it, sm.v[st], &sm.v_full[st]);
-          ++kv_count;
+        auto issue_k = [&](int t) -> bool {
+          const uint32_t st = k_issued % K_STAGES, use = k_issued / K_STAGES;
+          if (use > 0 && !mbar_wait(&sm.k_empty[st], (use - 1) & 1, abort)) return false;
+          issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, false, __ldg(tiles + it.tile0 + t), it, sm.k[st],
+                   &sm.k_full[st]);
+          ++k_issued;
+          return true;
+        };
+        auto issue_v = [&](int t) -> bool {
+          const uint32_t st = v_issued % V_STAGES, use = v_issued / V_STAGES;
+          if (use > 0 && !mbar_wait(&sm.v_empty[st], (use - 1) & 1, abort)) return false;
+          issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, true, __ldg(tiles + it.tile0 + t), it, sm.v[st],
+                   &sm.v_full[st]);
+          ++v_issued;
+          return true;
+        };
+        const int lead = min(K_STAGES - 1, it.ntiles);
+        for (int t = 0; t < lead && ok; ++t) ok = issue_k(t);
+        for (int t = 0; t < it.ntiles && ok; ++t) {
+          if (t + lead < it.ntiles) ok = issue_k(t + lead);
+          if (ok) ok = issue_v(t);
         }
       }
       if (!ok) {
         // let the copies already issued land before the CTA goes away
-        for (uint32_t c = (kv_count > KV_STAGES ? kv_count - KV_STAGES : 0); c < kv_count; ++c) {
-          const uint32_t st = c % KV_STAGES, use = c / KV_STAGES;
-          mbar_wait(&sm.k_full[st], use & 1, abort, 100000000ull);
-          mbar_wait(&sm.v_full[st], use & 1, abort, 100000000ull);
-        }
+        for (uint32_t c = (k_issued > K_STAGES ? k_issued - K_STAGES : 0); c < k_issued; ++c)
+          mbar_wait(&sm.k_full[c % K_STAGES], (c / K_STAGES) & 1, abort, 100000000ull);
+        for (uint32_t c = (v_issued > V_STAGES ? v_issued - V_STAGES : 0); c < v_issued; ++c)
+          mbar_wait(&sm.v_full[c % V_STAGES], (c / V_STAGES) & 1, abort, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -325,7 +352,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
       const uint32_t q_addr = smem_addr(sm.q), p_addr = smem_addr(sm.p);
-      uint32_t kv_count = 0, pv_count = 0, s_count = 0, q_uses = 0, p_uses = 0, items_done = 0;
+      uint32_t k_used = 0, v_used = 0, s_count = 0, q_uses = 0, p_uses = 0, items_done = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         ItemInfo it;
@@ -333,7 +360,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (!mbar_wait(&sm.q_full, q_uses & 1, abort)) { ok = false; break; }
         ++q_uses;
         auto do_pv = [&](int t) -> bool {
-          const uint32_t st = pv_count % KV_STAGES, use = pv_count / KV_STAGES;
+          const uint32_t st = v_used % V_STAGES, use = v_used / V_STAGES;
           if (!mbar_wait(&sm.v_full[st], use & 1, abort)) return false;
           if (t == 0 && items_done > 0 && !mbar_wait(&sm.o_free, (items_done - 1) & 1, abort)) return false;
           const uint32_t v_addr = smem_addr(sm.v[st]);
@@ -351,11 +378,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           }
           ++p_uses;
           umma_commit(&sm.v_empty[st]);
-          ++pv_count;
+          ++v_used;
           return true;
         };
         for (int t = 0; t < it.ntiles && ok; ++t) {
-          const uint32_t st = kv_count % KV_STAGES, use = kv_count / KV_STAGES;
+          const uint32_t st = k_used % K_STAGES, use = k_used / K_STAGES;
           const uint32_t sb = s_count & 1, su = s_count >> 1;
           if (!mbar_wait(&sm.k_full[st], use & 1, abort)) { ok = false; break; }
           if (su > 0 && !mbar_wait(&sm.s_free[sb], (su - 1) & 1, abort)) { ok = false; break; }
@@ -370,7 +397,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           umma_commit(&sm.s_full[sb]);
           umma_commit(&sm.k_empty[st]);
           if (t == it.ntiles - 1) umma_commit(&sm.q_empty);
-          ++kv_count;
+          ++k_used;
           ++s_count;
           if (t > 0 && !do_pv(t - 1)) { ok = false; break; }
         }
@@ -442,27 +469,30 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (!mbar_wait(&sm.s_full[sb], su & 1, abort)) { ok = false; break; }
         tc_fence_after();
         float s[64];
-        const uint32_t scol = lane_base + (sb ? TM_S1 : TM_S0) + 64 * g;
+        {
+          const uint32_t scol = lane_base + (sb ? TM_S1 : TM_S0) + 64 * g;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(scol + 32 * c, rr);
-          tmem_wait_ld();
+          for (int c = 0; c < 2; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(scol + 32 * c, rr);
+            tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) s[32 * c + j] = __uint_as_float(rr[j]);
+            for (int j = 0; j < 32; ++j) s[32 * c + j] = __uint_as_float(rr[j]);
+          }
         }
         tc_fence_before();
         mbar_arrive(&sm.s_free[sb]);
         ++s_count;
 
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float x = ((mk[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
-          s[c] = x;
-          mx4[c & 3] = fmaxf(mx4[c & 3], x);
+        for (int c = 0; c < 64; ++c) s[c] = ((mk[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], s[c + 2 * q], s[c + 2 * q + 1]);
         }
-        const float mxs = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
+        const float mxs = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * p.scale_log2;
         float alpha = 1.f;
         bool resc = false;
         if (mxs > m_used + 8.f) {  // also true on the first finite max
@@ -470,6 +500,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           m_used = mxs;
           resc = true;
         }
+
         // the previous P_g V_g must be complete before P_g is overwritten or O_g rescaled
         if (tt > 0) {
           if (!mbar_wait(&sm.pv_done[g], pv_waits & 1, abort)) { ok = false; break; }
@@ -519,17 +550,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // epilogue: both halves' last P V done, then O = (c0 O_0 + c1 O_1) / (c0 l0 + c1 l1)
       if (!mbar_wait(&sm.pv_done[g], pv_waits & 1, abort)) { ok = false; break; }
       ++pv_waits;
-      const int ip = items_done & 1;
-      sm.xm[ip][g][t] = m_used;
-      sm.xl[ip][g][t] = l;
+      sm.xm[g][t] = m_used;
+      sm.xl[g][t] = l;
       tc_fence_before();
       named_bar_sync(1, 256);
       tc_fence_after();
-      const float m0 = sm.xm[ip][0][t], m1 = sm.xm[ip][1][t];
+      const float m0 = sm.xm[0][t], m1 = sm.xm[1][t];
       const float M = fmaxf(m0, m1);
       const float c0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M);
       const float c1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
-      const float ltot = c0 * sm.xl[ip][0][t] + c1 * sm.xl[ip][1][t];
+      const float ltot = c0 * sm.xl[0][t] + c1 * sm.xl[1][t];
+      named_bar_sync(1, 256);  // both halves read before the next item's values land
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
       const float f0 = c0 * inv, f1 = c1 * inv;
       uint4* dst = reinterpret_cast<uint4*>(op + orow);
@@ -630,7 +661,7 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
   p.n_items = dp.n_items;
   p.scale_log2 = dp.scale * 1.4426950408889634f;
   p.lse = lse;
-  const size_t smem = sizeof(AttnSmem) + 1024;
+  const size_t smem = sizeof(AttnSmem);
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(msa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
