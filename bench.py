@@ -157,6 +157,20 @@ def cores():
     return len(os.sched_getaffinity(0))
 
 
+def job_totals(elapsed_ms: float, flops: float, world: int, device=None):
+    """Max of the timed region over ranks and the sum of executed FLOPs over ranks (each rank
+    runs its own layer: weak scaling).  A collective only on these two scalars."""
+    if world <= 1:
+        return float(elapsed_ms), float(flops)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(elapsed_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    f = torch.tensor([float(flops)], dtype=torch.float64, device=device)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(f.item())
+
+
 # ---------------------------------------------------------------------------------------
 def make_host_inputs(p, seed):
     Q, K, V = workload.make_inputs(p, seed=seed)
@@ -252,15 +266,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = start.elapsed_time(end)
     stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # ms
     # max over ranks of the timed region; sum of executed FLOPs over ranks
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        f = torch.tensor([float(exec_flops)], device=dev, dtype=torch.float64)
-        dist.all_reduce(f, op=dist.ReduceOp.SUM)
-        job_flops = float(f.item())
-    else:
-        job_flops = float(exec_flops)
+    total_ms, job_flops = job_totals(total_ms, exec_flops, world, dev)
     ms_step = total_ms / args.steps
     value = job_flops * args.steps / (total_ms * 1e-3) / 1e12
 
@@ -289,11 +295,7 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         s1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = s0.elapsed_time(s1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms, _ = job_totals(s0.elapsed_time(s1), 0.0, world, dev)
         bi = (Qh.nbytes + Kh.nbytes + Vh.nbytes)
         bo = int(np.prod(o.shape)) * 2
         e2e = {"value": job_flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
