@@ -75,6 +75,7 @@ def _load():
         "msa_device_status": ([_P, _P, _P], _I32),
         "msa_status_string": ([_I32], ctypes.c_char_p),
         "msa_kernel_launches": ([], ctypes.c_uint64),
+        "msa_vslash_estimate_static": ([_P, _P, _I64, _I64, _I64, _F32, _I32, _I32, _P, _P, _P, _P], _I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -86,7 +87,8 @@ def _load():
 _lib = _load()
 EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_estimate", "msa_set_indices",
            "msa_permute", "msa_sparse_prefill", "msa_unpermute", "msa_read_indices", "msa_read_tiles",
-           "msa_tile_stats", "msa_device_status", "msa_status_string", "msa_kernel_launches")
+           "msa_tile_stats", "msa_device_status", "msa_status_string", "msa_kernel_launches",
+           "msa_vslash_estimate_static")
 
 
 def kernel_launches() -> int:
@@ -311,6 +313,17 @@ class Plan:
 
     def device_status(self, ws, stream=None) -> int:
         return int(_lib.msa_device_status(self._h, ws.data_ptr(), _stream_ptr(stream)))
+
+
+def vslash_estimate_static(Qh, Kh, scale: float, k_v: int, k_s: int, v_out, s_out, counts_out, stream=None):
+    """msa_vslash_estimate_static: vertical/slash lines of one head without any workspace.
+    Qh, Kh: [L, 128] bf16 CUDA tensors; v_out [k_v], s_out [k_s], counts_out [2]: int32 CUDA
+    tensors the caller allocated beforehand."""
+    assert Qh.dim() == 2 and Kh.dim() == 2 and Qh.stride(1) == 1 and Kh.stride(1) == 1
+    _check("msa_vslash_estimate_static",
+           _lib.msa_vslash_estimate_static(Qh.data_ptr(), Kh.data_ptr(), Qh.shape[0], Qh.stride(0), Kh.stride(0),
+                                           float(scale), int(k_v), int(k_s), v_out.data_ptr(), s_out.data_ptr(),
+                                           counts_out.data_ptr(), _stream_ptr(stream)))
 
 
 def executed_flops(tiles: int) -> int:

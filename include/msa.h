@@ -207,6 +207,30 @@ msa_status msa_device_status(const msa_plan* plan, void* ws, void* stream);
 
 const char* msa_status_string(msa_status status);
 
+/* ---- allocation-free variant ----
+ *
+ * Vertical-slash index estimation of ONE query head (the vertical and slash lines of its last
+ * 64 queries, exactly as msa_estimate computes them for a vertical-slash head) for callers
+ * that cannot allocate device memory or provide a workspace: code running inside another
+ * framework's memory manager, or serving loops where cudaMalloc and its implicit device
+ * synchronisation are not allowed.  This call has no counterpart in the method's description;
+ * it exists for those callers.
+ *  - Inputs: Q and K of the head, bf16 [L][128] on the device with row strides q_row_stride /
+ *    k_row_stride (elements, multiples of 8; pointers 16-byte aligned); softmax scale.
+ *  - Outputs (device, caller-owned): v_out[k_v] vertical-line key positions and s_out[k_s]
+ *    slash-line offsets, each ascending; counts_out[2] = number written to each.
+ *  - Scratch: a fixed 1.1 MB array compiled into the library (every GPU that loads libmsa.so
+ *    holds it until the process exits); L must be a multiple of 64 and at most 65536, larger L
+ *    returns MSA_ERR_UNSUPPORTED; k_v, k_s in [1, L].
+ *  - The first call on a device looks up the array's device address (a runtime call, no
+ *    allocation); make that first call before any stream capture on that device.
+ *  - Every call shares the one array and keeps its last contents: calls that may overlap on the
+ *    GPU (different streams, or different threads) race and must be serialised by the caller.
+ *  - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating library routine. */
+msa_status msa_vslash_estimate_static(const void* Q, const void* K, int64_t L, int64_t q_row_stride,
+                                      int64_t k_row_stride, float scale, int32_t k_v, int32_t k_s, int32_t* v_out,
+                                      int32_t* s_out, int32_t* counts_out, void* stream);
+
 /* Number of CUDA kernels this library has launched since it was loaded (all plans, all
  * threads); lets a caller count the kernels of one call by differencing. */
 uint64_t msa_kernel_launches(void);
