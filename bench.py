@@ -346,6 +346,53 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """The budget sweep on the LLaMA-3-8B-shaped layer: one JSON line per (L, budget), with the
+    estimation time against the attention time.  Not the benchmark line: a table."""
+    import torch
+    import dynamic_sparse_attention_head_b200 as msa
+    lengths = [int(x) for x in args.sweep_lengths.split(",")]
+    budgets = [None if x == "dense" else float(x) for x in args.sweep_budgets.split(",")]
+    for L in lengths:
+        for b in budgets:
+            p = workload.sweep_layer(L, b)
+            Qh, Kh, Vh = make_host_inputs(p, seed=0)
+            q, k, v = (torch.from_numpy(x).view(torch.bfloat16).cuda() for x in (Qh, Kh, Vh))
+            del Qh, Kh, Vh
+            o = torch.empty_like(q)
+            plan = msa.Plan(p)
+            ws = plan.alloc_workspace()
+            st = torch.cuda.current_stream()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            stages = []
+            for i in range(args.warmup + args.steps):
+                ev[0].record(st)
+                plan.estimate(q, k, ws)
+                ev[1].record(st)
+                plan.permute(q, k, v, ws)
+                ev[2].record(st)
+                plan.sparse_prefill(q, k, v, ws)
+                ev[3].record(st)
+                plan.unpermute(ws, o)
+                ev[4].record(st)
+                torch.cuda.synchronize()
+                if i >= args.warmup:
+                    stages.append([ev[j].elapsed_time(ev[j + 1]) for j in range(4)])
+            assert plan.device_status(ws) == 0
+            tiles, _ = plan.tile_stats(ws)
+            st_ms = np.mean(np.array(stages), axis=0)
+            flops = msa.executed_flops(tiles)
+            print(json.dumps({"sweep": "llama3-8b-text", "L": L, "budget": b, "ms_per_layer": float(st_ms.sum()),
+                              "estimate_ms": float(st_ms[0]), "permute_ms": float(st_ms[1]),
+                              "attention_ms": float(st_ms[2]), "unpermute_ms": float(st_ms[3]),
+                              "estimate_over_attention": float(st_ms[0] / st_ms[2]),
+                              "executed_flops": flops, "dense_causal_flops": dense_causal_flops(p),
+                              "density": flops / dense_causal_flops(p),
+                              "attn_tflops": flops / (st_ms[2] * 1e-3) / 1e12}), flush=True)
+            del q, k, v, o, ws, plan
+            torch.cuda.empty_cache()
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm: bounded samples of the same workload on host cores."""
     if rank != 0:
@@ -411,7 +458,13 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=32)
+    ap.add_argument("--sweep", action="store_true", help="budget sweep table instead of the benchmark line")
+    ap.add_argument("--sweep-lengths", default=",".join(str(x) for x in workload.SWEEP_LENGTHS))
+    ap.add_argument("--sweep-budgets", default="0.02,0.05,0.1,0.25,dense")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

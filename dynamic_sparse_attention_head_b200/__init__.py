@@ -288,6 +288,8 @@ class Plan:
         return out
 
     def read_tiles(self, head: int, ws, stream=None) -> List[Dict]:
+        """Work list of one head: per item its class, rows and tiles (source, the 128 key
+        positions, and whether the tile is flagged fully allowed for every row)."""
         r = self._record(_lib.msa_read_tiles, head, ws, stream)
         n_items, i = int(r[0]), 1
         items = []
@@ -302,7 +304,7 @@ class Plan:
                 src = int(r[i])
                 keys = r[i + 1:i + 1 + 128].astype(np.int64)
                 i += 129
-                tiles.append((src, keys))
+                tiles.append((src & 7, keys, bool(src & 8)))
             items.append({"cls": cls, "nrows": nrows, "rows": rows, "tiles": tiles})
         return items
 

@@ -3,16 +3,19 @@
 // MMInference ("key machinery"): block-sparse FlashAttention-style kernels load only the
 // permuted blocks and keep the tensor-core compute dense; "Grid-Shape Flash Attention"
 // (Algorithm 5) is the FlashAttention-2 online softmax over those blocks.  Here:
-//  - one persistent CTA per SM walks 128-query work items;
-//  - warp 0 streams Q, K and V tiles with TMA (128-byte swizzle) into a 2-stage ring;
-//  - warp 1 (one elected thread) issues tcgen05.mma: S = Q K^T into one of two TMEM
-//    buffers, then O += P V with O resident in TMEM for the whole work item;
-//  - warps 2..9 form two warpgroups, each owning TMEM lanes 0..127 (one query row per thread)
-//    and one 64-key half of every tile: they read S with
-//    tcgen05.ld, apply the element mask (causal in original positions + the head's
-//    pattern), run the online softmax in fp32 (exp2 on MUFU, lazy rescale of O when the
-//    running max grows by more than 2^8), write P as bf16 into shared memory in the
-//    K-major 128B-swizzled layout the MMA reads, and finally normalise O.
+//  - one persistent CTA per SM runs two independent streams of 128-query work items
+//    (stream s takes items 2 b + s, 2 b + s + 2 G, ... of CTA b in a grid of G);
+//  - warps 0 and 2 stream the Q, K and V tiles of stream 0 and 1 with TMA (128-byte
+//    swizzle) into single-buffered slots of their own;
+//  - warps 1 and 3 (one thread each) issue the tcgen05.mma of stream 0 and 1:
+//    S_s = Q_s K^T into stream s's TMEM columns, then O_s += P_s V with P_s read from TMEM
+//    and O_s resident in TMEM for the whole work item.  While one stream's softmax runs, the
+//    tensor core works on the other stream;
+//  - warps 4..7 (stream 0) and 8..11 (stream 1) each own TMEM lanes 0..127, one query row per
+//    thread and all 128 keys of every tile: they read S with tcgen05.ld, apply the element
+//    mask (causal in original positions + the head's pattern), run the online softmax in fp32
+//    (exp2 on MUFU, lazy rescale of O when the running max grows by more than 2^8), write P
+//    as packed bf16 over the first 64 columns of S with tcgen05.st, and finally normalise O.
 // Every wait is bounded; on a timeout the CTA records DEV_ERR_TIMEOUT and unwinds.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -38,32 +41,38 @@ struct AttnParams {
   float* lse;              // [Hq][L] or null
 };
 
-constexpr int ATT_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (two warpgroups)
-constexpr int K_STAGES = 2;  // K tiles are loaded ahead of V tiles
-constexpr int V_STAGES = 2;
+// warpgroup 0: warps 0 / 2 TMA of stream 0 / 1, warps 1 / 3 MMA of stream 0 / 1; warpgroups
+// 1 / 2: softmax of stream 0 / 1
+constexpr int ATT_THREADS = 384;
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512), warpgroup 0 gives
+// back to 72 and the softmax warpgroups grow to 216: 128 x 72 + 256 x 216 = 64512.
+constexpr int REG_CTRL = 72, REG_SOFTMAX = 216;
+static_assert(128 * REG_CTRL + 256 * REG_SOFTMAX <= ATT_THREADS * 168, "register split exceeds the launch allocation");
+constexpr int N_STREAMS = 2;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // one 128x128 bf16 tile
 constexpr uint32_t ATOM_BYTES = 128 * 128;      // one [128 rows][64 cols] 128B-swizzled atom
 
 struct __align__(1024) AttnSmem {
-  uint8_t q[TILE_BYTES];
-  uint8_t k[K_STAGES][TILE_BYTES];
-  uint8_t v[V_STAGES][TILE_BYTES];
-  uint8_t p[TILE_BYTES];
-  uint64_t q_full, q_empty;
-  uint64_t k_full[K_STAGES], k_empty[K_STAGES];
-  uint64_t v_full[V_STAGES], v_empty[V_STAGES];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], pv_done[2], o_free, drain;
-  float xm[2][128];  // [key half][row] running max of the half (log2 units)
-  float xl[2][128];  // [key half][row] running sum of the half
+  uint8_t q[N_STREAMS][TILE_BYTES];
+  uint8_t k[N_STREAMS][TILE_BYTES];
+  uint8_t v[N_STREAMS][TILE_BYTES];
+  uint64_t q_full[N_STREAMS], q_empty[N_STREAMS];
+  uint64_t k_full[N_STREAMS], k_empty[N_STREAMS];
+  uint64_t v_full[N_STREAMS], v_empty[N_STREAMS];
+  uint64_t s_full[N_STREAMS], p_full[N_STREAMS];
+  uint64_t o_full[N_STREAMS], o_free[N_STREAMS];
+  uint64_t drain[N_STREAMS];
   uint32_t tmem_base;
   int abort;
+  int issue_lock;
 };
 
 static_assert(sizeof(AttnSmem) <= 232448, "attention shared memory exceeds 227 KB per CTA");
 
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;  // O of key half g at TM_O + 128 g
+// stream s: S (fp32, 128 columns; P as packed bf16 pairs over its first 64) at 256 s,
+// O (fp32, 128 columns) at 256 s + 128
+constexpr uint32_t TM_STREAM = 256, TM_OOFF = 128;
 
 __device__ __forceinline__ const ClassStatic& class_of(const AttnParams& p, int c) {
   return reinterpret_cast<const ClassStatic*>(p.ws + p.lay.classes)[c];
@@ -99,6 +108,13 @@ __device__ __forceinline__ bool load_item(const AttnParams& p, int item, ItemInf
   return it.ntiles >= 0;
 }
 
+// Advances `item` (in steps of `stride`) to the next item with at least one tile.
+__device__ __forceinline__ bool next_work(const AttnParams& p, int& item, int stride, ItemInfo& it) {
+  for (; item < p.n_items; item += stride)
+    if (load_item(p, item, it) && it.ntiles > 0) return true;
+  return false;
+}
+
 // Per-row state of the element mask.
 struct RowCtx {
   int valid, qpos, qcoord;
@@ -109,107 +125,106 @@ struct RowCtx {
   const int32_t* xpos;
 };
 
-__device__ __forceinline__ void prefix_mask2(uint32_t (&m)[2], int n) {
-#pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    int k = n - 32 * w;
-    m[w] = k >= 32 ? 0xFFFFFFFFu : (k <= 0 ? 0u : ((1u << k) - 1u));
-  }
+// Bits [0, n) of the 32-column word w of a 128-column row (n clipped to [0, 128]).
+__device__ __forceinline__ uint32_t low_bits(int n, int w) {
+  const int k = n - 32 * w;
+  return k >= 32 ? 0xFFFFFFFFu : (k <= 0 ? 0u : ((1u << k) - 1u));
 }
 
-// Mask words of one query row against key columns [64 half, 64 half + 64) of a tile, in two
-// steps so the bitmap loads of the next tile are in flight while the current tile is
-// processed: mask_prefetch issues the loads, mask_finish combines them.
+__device__ __forceinline__ void prefix_mask4(uint32_t (&m)[4], int n) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) m[w] = low_bits(n, w);
+}
+
+// Mask words of one query row against the 128 key columns of a tile, in two steps so the
+// bitmap loads are in flight while the thread waits for S: mask_prefetch issues the loads,
+// mask_finish combines them.
 struct MaskRaw {
   int src, krow, kc0;
-  uint32_t sl[3], ex[3], bk0, bk1;
+  uint32_t sl[5], ex[5], bk[3];
 };
 
 __device__ __forceinline__ uint32_t ldg_word(const uint32_t* bm, int nwords, int w) {
   return (w >= 0 && w < nwords) ? __ldg(bm + w) : 0u;
 }
 
-__device__ __forceinline__ void mask_prefetch(const RowCtx& rc, uint32_t tile, int half, MaskRaw& r) {
+__device__ __forceinline__ void mask_prefetch(const RowCtx& rc, uint32_t tile, MaskRaw& r) {
   r.src = (int)(tile >> 28);
-  r.krow = (int)(tile & 0x0FFFFFFFu);
-  r.kc0 = rc.kc_lo + (r.krow - rc.krow_lo) + 64 * half;
+  r.krow = (int)(tile & TILE_ROW_MASK);
+  r.kc0 = rc.kc_lo + (r.krow - rc.krow_lo);
   if (!rc.valid || r.src == SRC_X) return;
   if (rc.flags & CF_SLASH) {
-    const int w0 = (rc.qcoord - r.kc0 - 63) >> 5;
+    const int w0 = (rc.qcoord - r.kc0 - 127) >> 5;
 #pragma unroll
-    for (int i = 0; i < 3; ++i) r.sl[i] = ldg_word(rc.slash, rc.nwords, w0 + i);
+    for (int i = 0; i < 5; ++i) r.sl[i] = ldg_word(rc.slash, rc.nwords, w0 + i);
   }
   if (rc.flags & CF_EXCL) {
     const int w0 = r.kc0 >> 5;
 #pragma unroll
-    for (int i = 0; i < 3; ++i) r.ex[i] = ldg_word(rc.excl, rc.nwords, w0 + i);
+    for (int i = 0; i < 5; ++i) r.ex[i] = ldg_word(rc.excl, rc.nwords, w0 + i);
   }
   if (rc.flags & CF_BLOCK) {
     const uint32_t* row = rc.blk + (size_t)(rc.qcoord >> 6) * rc.blk_wpr;
     const int nbk = (rc.kc_hi + 63) >> 6;
-    const int b0 = r.kc0 >> 6, b1 = b0 + 1;  // a 64-column half touches at most two blocks
-    r.bk0 = b0 < nbk ? (__ldg(row + (b0 >> 5)) >> (b0 & 31)) & 1u : 0u;
-    r.bk1 = b1 < nbk ? (__ldg(row + (b1 >> 5)) >> (b1 & 31)) & 1u : 0u;
+    const int b0 = r.kc0 >> 6;  // 128 columns touch at most three 64-blocks
+#pragma unroll
+    for (int i = 0; i < 3; ++i) r.bk[i] = (b0 + i) < nbk ? (__ldg(row + ((b0 + i) >> 5)) >> ((b0 + i) & 31)) & 1u : 0u;
   }
 }
 
-__device__ __forceinline__ void mask_finish(const RowCtx& rc, const MaskRaw& r, int half, uint32_t (&m)[2]) {
+__device__ __forceinline__ void mask_finish(const RowCtx& rc, const MaskRaw& r, uint32_t (&m)[4]) {
   if (!rc.valid) {
-    m[0] = m[1] = 0u;
+    m[0] = m[1] = m[2] = m[3] = 0u;
     return;
   }
   if (r.src == SRC_X) {
     // gathered keys are sorted by position: the allowed ones are a prefix
-    const int32_t* kp = rc.xpos + (r.krow - rc.x_row0) + 64 * half;
-    int lo = 0, hi = 64;
+    const int32_t* kp = rc.xpos + (r.krow - rc.x_row0);
+    int lo = 0, hi = 128;
     while (lo < hi) {
       int mid = (lo + hi) >> 1;
       if (__ldg(kp + mid) <= rc.qpos) lo = mid + 1;
       else hi = mid;
     }
-    prefix_mask2(m, lo);
+    prefix_mask4(m, lo);
     return;
   }
   const int kc0 = r.kc0;
-  prefix_mask2(m, min(rc.qcoord - kc0 + 1, rc.kc_hi - kc0));  // causal and inside the region
+  prefix_mask4(m, min(rc.qcoord - kc0 + 1, rc.kc_hi - kc0));  // causal and inside the region
   if (!(rc.flags & CF_DENSE)) {
-    uint32_t any[2] = {0u, 0u};
+    uint32_t any[4] = {0u, 0u, 0u, 0u};
     if (rc.flags & CF_SINK) {
-      uint32_t t[2];
-      prefix_mask2(t, rc.sink - kc0);
-      any[0] |= t[0];
-      any[1] |= t[1];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) any[w] |= low_bits(rc.sink - kc0, w);
     }
-    if (rc.flags & CF_BAND) {
-      uint32_t t[2];
-      prefix_mask2(t, rc.qcoord - rc.band + 1 - kc0);  // columns below qcoord - band + 1 are outside
-      any[0] |= ~t[0];
-      any[1] |= ~t[1];
+    if (rc.flags & CF_BAND) {  // columns below qcoord - band + 1 are outside the band
+#pragma unroll
+      for (int w = 0; w < 4; ++w) any[w] |= ~low_bits(rc.qcoord - rc.band + 1 - kc0, w);
     }
     if (rc.flags & CF_SLASH) {
-      // column c has offset qcoord - kc0 - c: bits [base, base + 64) reversed
-      const int sh = (rc.qcoord - kc0 - 63) & 31;
-      const uint32_t b0 = __funnelshift_r(r.sl[0], r.sl[1], sh), b1 = __funnelshift_r(r.sl[1], r.sl[2], sh);
-      any[0] |= __brev(b1);
-      any[1] |= __brev(b0);
+      // column c has offset qcoord - kc0 - c: bits [base, base + 128) of the offset bitmap,
+      // base = qcoord - kc0 - 127, in reverse column order
+      const int sh = (rc.qcoord - kc0 - 127) & 31;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) any[w] |= __brev(__funnelshift_r(r.sl[3 - w], r.sl[4 - w], sh));
     }
     if (rc.flags & CF_BLOCK) {
-      // columns before the next 64-boundary of the coordinate lie in block kc0 >> 6
+      // columns [0, split) lie in block kc0 >> 6, [split, split + 64) in the next one, the
+      // rest in the one after
       const int split = 64 - (kc0 & 63);
 #pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        const int lo = split - 32 * w;  // columns of word w inside the first block
-        const uint32_t low = lo >= 32 ? 0xFFFFFFFFu : (lo <= 0 ? 0u : ((1u << lo) - 1u));
-        any[w] |= (r.bk0 ? low : 0u) | (r.bk1 ? ~low : 0u);
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t a = low_bits(split, w), b = low_bits(split + 64, w);
+        any[w] |= (r.bk[0] ? a : 0u) | (r.bk[1] ? (b & ~a) : 0u) | (r.bk[2] ? ~b : 0u);
       }
     }
-    m[0] &= any[0];
-    m[1] &= any[1];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) m[w] &= any[w];
   }
   if (rc.flags & CF_EXCL) {
     const int sh = kc0 & 31;
-    m[0] &= ~__funnelshift_r(r.ex[0], r.ex[1], sh);
-    m[1] &= ~__funnelshift_r(r.ex[1], r.ex[2], sh);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) m[w] &= ~__funnelshift_r(r.ex[w], r.ex[w + 1], sh);
   }
 }
 
@@ -219,16 +234,12 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 __device__ __forceinline__ void issue_kv(const CUtensorMap* tk, const CUtensorMap* tv, const CUtensorMap* tk2,
                                          const CUtensorMap* tv2, const CUtensorMap* txk, const CUtensorMap* txv,
                                          bool is_v, uint32_t tile, const ItemInfo& it, uint8_t* dst,
                                          uint64_t* bar) {
   const int src = (int)(tile >> 28);
-  const int row = (int)(tile & 0x0FFFFFFFu);
+  const int row = (int)(tile & TILE_ROW_MASK);
   const CUtensorMap* m;
   int c2;
   if (src == SRC_X) {
@@ -244,6 +255,104 @@ __device__ __forceinline__ void issue_kv(const CUtensorMap* tk, const CUtensorMa
   mbar_arrive_expect_tx(bar, TILE_BYTES);
   tma_load_3d(dst, m, bar, 0, row, c2);
   tma_load_3d(dst + ATOM_BYTES, m, bar, 64, row, c2);
+}
+
+// No-progress guard of the polling roles: true (and *abort raised) after one second without
+// progress, or as soon as another role has aborted.
+struct Watchdog {
+  uint64_t t0 = 0;
+  int idle = 0;
+  __device__ __forceinline__ void progress() { idle = 0; }
+  __device__ __forceinline__ bool expired(volatile int* abort) {
+    if (++idle < 64) return false;
+    if (idle == 64) t0 = global_ns();
+    if (*abort) return true;
+    if (global_ns() - t0 > 1000000000ull) {
+      *abort = 1;
+      return true;
+    }
+    return false;
+  }
+};
+
+// Exclusive right to issue tcgen05.mma, held for one group at a time (see mma_stream).
+__device__ __forceinline__ bool issue_lock(int* lock, volatile int* abort) {
+  if (atomicCAS(lock, 0, 1) == 0) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    for (int i = 0; i < 32; ++i)
+      if (atomicCAS(lock, 0, 1) == 0) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > 1000000000ull) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void issue_unlock(int* lock) { atomicExch(lock, 0); }
+
+// MMA issuer of one stream (one thread).  Per item: QK(0), then the groups [PV(j), QK(j + 1)]
+// and finally PV(n - 1).  QK(j + 1) may overwrite P(j) in TMEM because the tcgen05.mma
+// operations of one thread run in issue order.  Each stream has its own issuer, so one
+// stream never waits for the other's softmax; a group is issued under a lock shared by the two
+// issuers, so the tensor pipe receives whole groups back to back instead of interleaved.  A
+// stream whose group follows the other's gets its S one group later and starts its softmax
+// then: the streams settle half a cycle apart, and one stream's MMAs run while the other
+// computes its softmax.
+__device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, uint32_t tmem, int s, int stride,
+                                           volatile int* abort) {
+  constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
+  const uint32_t s_col = tmem + TM_STREAM * s;
+  uint32_t q_use = 0, k_use = 0, v_use = 0, done = 0;
+  auto qk = [&](bool last) {
+    tc_fence_after();
+    uint32_t q_addr = smem_addr(sm.q[s]), k_addr = smem_addr(sm.k[s]);
+    // keep the descriptors from being hoisted out of the loop: the issuer has 72 registers
+    asm volatile("" : "+r"(q_addr), "+r"(k_addr));
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t off = (kk >> 2) * ATOM_BYTES + (kk & 3) * 32;
+      umma_ss(s_col, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK,
+              kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&sm.s_full[s]);
+    umma_commit(&sm.k_empty[s]);
+    if (last) umma_commit(&sm.q_empty[s]);
+    ++k_use;
+  };
+  ItemInfo it;
+  for (int item = N_STREAMS * blockIdx.x + s; next_work(p, item, stride, it); item += stride) {
+    const int n = it.ntiles;
+    if (!mbar_wait(&sm.q_full[s], q_use & 1, abort)) return;
+    ++q_use;
+    if (!mbar_wait(&sm.k_full[s], k_use & 1, abort)) return;
+    if (!issue_lock(&sm.issue_lock, abort)) return;
+    qk(n == 1);
+    issue_unlock(&sm.issue_lock);
+    for (int j = 0; j < n; ++j) {
+      if (j == 0 && done > 0 && !mbar_wait(&sm.o_free[s], (done - 1) & 1, abort)) return;
+      if (!mbar_wait(&sm.v_full[s], v_use & 1, abort)) return;
+      if (!mbar_wait(&sm.p_full[s], v_use & 1, abort)) return;
+      if (j + 1 < n && !mbar_wait(&sm.k_full[s], k_use & 1, abort)) return;
+      if (!issue_lock(&sm.issue_lock, abort)) return;
+      tc_fence_after();
+      {  // O_s += P_s V_j
+        uint32_t v_addr = smem_addr(sm.v[s]);
+        asm volatile("" : "+r"(v_addr));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // 16 keys per step: 8 TMEM columns of P, 2 KB of V
+          umma_ts(s_col + TM_OOFF, s_col + 8 * kk, smem_desc_sw128(v_addr + kk * 2048, ATOM_BYTES, 1024), IDESC_PV,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&sm.v_empty[s]);
+      ++v_use;
+      if (j + 1 < n) qk(j + 2 == n);  // S_s = Q_s K_{j+1}^T
+      issue_unlock(&sm.issue_lock);
+    }
+    umma_commit(&sm.o_full[s]);
+    ++done;
+  }
 }
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
@@ -262,29 +371,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int lane = threadIdx.x & 31;
   volatile int* abort = &sm.abort;
   uint32_t* err = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.ws + p.lay.header));
+  const int stride = N_STREAMS * gridDim.x;
 
   if (threadIdx.x == 0) {
     sm.abort = 0;
-    mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_empty, 1);
-    for (int s = 0; s < K_STAGES; ++s) {
+    sm.issue_lock = 0;
+    for (int s = 0; s < N_STREAMS; ++s) {
+      mbar_init(&sm.q_full[s], 1);
+      mbar_init(&sm.q_empty[s], 1);
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
-    }
-    for (int s = 0; s < V_STAGES; ++s) {
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.p_full[s], 128);
+      mbar_init(&sm.o_full[s], 1);
+      mbar_init(&sm.o_free[s], 128);
+      mbar_init(&sm.drain[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 256);
-    }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&sm.p_full[g], 128);
-      mbar_init(&sm.pv_done[g], 1);
-    }
-    mbar_init(&sm.o_free, 256);
-    mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc<TMEM_COLS>(&sm.tmem_base);
@@ -293,135 +397,98 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp < 4) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_CTRL));
+   if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------------ TMA producers
+    // Warp 0 loads stream 0, warp 2 stream 1: two independent load sequences each, polled in
+    // turn: Q then the K tiles of every item (slot freed by the QK MMA), and the V tiles
+    // (slot freed by the PV MMA).
     if (lane == 0) {
+      const int s = warp >> 1;
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      uint32_t k_issued = 0, v_issued = 0, q_uses = 0;
       const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
-      bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        ItemInfo it;
-        if (!load_item(p, item, it) || it.ntiles == 0) continue;
-        if (q_uses > 0 && !mbar_wait(&sm.q_empty, (q_uses - 1) & 1, abort)) { ok = false; break; }
-        ++q_uses;
-        mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES);
-        if (it.q_src) {
-          tma_load_3d(sm.q, &tmQp, &sm.q_full, 0, it.qrow0 + it.row0, it.q_slice);
-          tma_load_3d(sm.q + ATOM_BYTES, &tmQp, &sm.q_full, 64, it.qrow0 + it.row0, it.q_slice);
-        } else {
-          tma_load_3d(sm.q, &tmQ, &sm.q_full, 0, it.row0, it.head);
-          tma_load_3d(sm.q + ATOM_BYTES, &tmQ, &sm.q_full, 64, it.row0, it.head);
-        }
-        auto issue_k = [&](int t) -> bool {
-          const uint32_t st = k_issued % K_STAGES, use = k_issued / K_STAGES;
-          if (use > 0 && !mbar_wait(&sm.k_empty[st], (use - 1) & 1, abort)) return false;
-          issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, false, __ldg(tiles + it.tile0 + t), it, sm.k[st],
-                   &sm.k_full[st]);
-          ++k_issued;
-          return true;
-        };
-        auto issue_v = [&](int t) -> bool {
-          const uint32_t st = v_issued % V_STAGES, use = v_issued / V_STAGES;
-          if (use > 0 && !mbar_wait(&sm.v_empty[st], (use - 1) & 1, abort)) return false;
-          issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, true, __ldg(tiles + it.tile0 + t), it, sm.v[st],
-                   &sm.v_full[st]);
-          ++v_issued;
-          return true;
-        };
-        const int lead = min(K_STAGES - 1, it.ntiles);
-        for (int t = 0; t < lead && ok; ++t) ok = issue_k(t);
-        for (int t = 0; t < it.ntiles && ok; ++t) {
-          if (t + lead < it.ntiles) ok = issue_k(t + lead);
-          if (ok) ok = issue_v(t);
-        }
-      }
-      if (!ok) {
-        // let the copies already issued land before the CTA goes away
-        for (uint32_t c = (k_issued > K_STAGES ? k_issued - K_STAGES : 0); c < k_issued; ++c)
-          mbar_wait(&sm.k_full[c % K_STAGES], (c / K_STAGES) & 1, abort, 100000000ull);
-        for (uint32_t c = (v_issued > V_STAGES ? v_issued - V_STAGES : 0); c < v_issued; ++c)
-          mbar_wait(&sm.v_full[c % V_STAGES], (c / V_STAGES) & 1, abort, 100000000ull);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
-      const uint32_t q_addr = smem_addr(sm.q), p_addr = smem_addr(sm.p);
-      uint32_t k_used = 0, v_used = 0, s_count = 0, q_uses = 0, p_uses = 0, items_done = 0;
-      bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        ItemInfo it;
-        if (!load_item(p, item, it) || it.ntiles == 0) continue;
-        if (!mbar_wait(&sm.q_full, q_uses & 1, abort)) { ok = false; break; }
-        ++q_uses;
-        auto do_pv = [&](int t) -> bool {
-          const uint32_t st = v_used % V_STAGES, use = v_used / V_STAGES;
-          if (!mbar_wait(&sm.v_full[st], use & 1, abort)) return false;
-          if (t == 0 && items_done > 0 && !mbar_wait(&sm.o_free, (items_done - 1) & 1, abort)) return false;
-          const uint32_t v_addr = smem_addr(sm.v[st]);
-          // O_g += P[:, 64g:64g+64] V[64g:64g+64, :] for each key half g, as soon as its P is ready
-          for (int g = 0; g < 2; ++g) {
-            if (!mbar_wait(&sm.p_full[g], p_uses & 1, abort)) return false;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = smem_desc_sw128(p_addr + g * ATOM_BYTES + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(v_addr + g * 8192 + kk * 2048, ATOM_BYTES, 1024);
-              umma_ss(tmem + TM_O + 128 * g, ad, bd, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+      int qk_item = N_STREAMS * blockIdx.x + s, v_item = qk_item, qk_op = 0, v_j = 0;
+      ItemInfo qk_it, v_it;
+      bool qk_live = next_work(p, qk_item, stride, qk_it);
+      bool v_live = next_work(p, v_item, stride, v_it);
+      uint32_t q_iss = 0, k_iss = 0, v_iss = 0;
+      Watchdog wd;
+      while (qk_live || v_live) {
+        if (qk_live) {
+          if (qk_op == 0) {
+            if (q_iss == 0 || mbar_test(&sm.q_empty[s], (q_iss - 1) & 1)) {
+              mbar_arrive_expect_tx(&sm.q_full[s], TILE_BYTES);
+              if (qk_it.q_src) {
+                tma_load_3d(sm.q[s], &tmQp, &sm.q_full[s], 0, qk_it.qrow0 + qk_it.row0, qk_it.q_slice);
+                tma_load_3d(sm.q[s] + ATOM_BYTES, &tmQp, &sm.q_full[s], 64, qk_it.qrow0 + qk_it.row0, qk_it.q_slice);
+              } else {
+                tma_load_3d(sm.q[s], &tmQ, &sm.q_full[s], 0, qk_it.row0, qk_it.head);
+                tma_load_3d(sm.q[s] + ATOM_BYTES, &tmQ, &sm.q_full[s], 64, qk_it.row0, qk_it.head);
+              }
+              ++q_iss;
+              qk_op = 1;
+              wd.progress();
             }
-            umma_commit(&sm.pv_done[g]);
+          } else if (k_iss == 0 || mbar_test(&sm.k_empty[s], (k_iss - 1) & 1)) {
+            const int j = qk_op - 1;
+            issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, false, __ldg(tiles + qk_it.tile0 + j), qk_it, sm.k[s],
+                     &sm.k_full[s]);
+            ++k_iss;
+            wd.progress();
+            if (j + 1 == qk_it.ntiles) {
+              qk_item += stride;
+              qk_live = next_work(p, qk_item, stride, qk_it);
+              qk_op = 0;
+            } else {
+              qk_op = j + 2;
+            }
           }
-          ++p_uses;
-          umma_commit(&sm.v_empty[st]);
-          ++v_used;
-          return true;
-        };
-        for (int t = 0; t < it.ntiles && ok; ++t) {
-          const uint32_t st = k_used % K_STAGES, use = k_used / K_STAGES;
-          const uint32_t sb = s_count & 1, su = s_count >> 1;
-          if (!mbar_wait(&sm.k_full[st], use & 1, abort)) { ok = false; break; }
-          if (su > 0 && !mbar_wait(&sm.s_free[sb], (su - 1) & 1, abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t k_addr = smem_addr(sm.k[st]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * ATOM_BYTES + (kk & 3) * 32;
-            umma_ss(tmem + (sb ? TM_S1 : TM_S0), smem_desc_sw128(q_addr + off, 16, 1024),
-                    smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&sm.s_full[sb]);
-          umma_commit(&sm.k_empty[st]);
-          if (t == it.ntiles - 1) umma_commit(&sm.q_empty);
-          ++k_used;
-          ++s_count;
-          if (t > 0 && !do_pv(t - 1)) { ok = false; break; }
         }
-        if (ok && !do_pv(it.ntiles - 1)) ok = false;
-        ++items_done;
+        if (v_live && (v_iss == 0 || mbar_test(&sm.v_empty[s], (v_iss - 1) & 1))) {
+          issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, true, __ldg(tiles + v_it.tile0 + v_j), v_it, sm.v[s],
+                   &sm.v_full[s]);
+          ++v_iss;
+          wd.progress();
+          if (++v_j == v_it.ntiles) {
+            v_item += stride;
+            v_live = next_work(p, v_item, stride, v_it);
+            v_j = 0;
+          }
+        }
+        if (wd.expired(abort)) {
+          // let the copies already issued land before the CTA goes away
+          if (q_iss) mbar_wait(&sm.q_full[s], (q_iss - 1) & 1, abort, 100000000ull);
+          if (k_iss) mbar_wait(&sm.k_full[s], (k_iss - 1) & 1, abort, 100000000ull);
+          if (v_iss) mbar_wait(&sm.v_full[s], (v_iss - 1) & 1, abort, 100000000ull);
+          break;
+        }
       }
-      // wait for every MMA issued by this thread before the tensor memory is released
-      umma_commit(&sm.drain);
-      mbar_wait(&sm.drain, 0, abort, 100000000ull);
     }
+   } else {
+    // ------------------------------------------------------------------ MMA issuers
+    // warp 1: stream 0, warp 3: stream 1
+    if (lane == 0) {
+      mma_stream(p, sm, tmem, warp >> 1, stride, abort);
+      // wait for every MMA issued by this thread before the tensor memory is released
+      umma_commit(&sm.drain[warp >> 1]);
+      mbar_wait(&sm.drain[warp >> 1], 0, abort, 100000000ull);
+    }
+   }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
     // ------------------------------------------------------------------ softmax / epilogue
-    // Two independent warpgroups: warpgroup g owns key columns [64g, 64g + 64) of every S
-    // tile with its own running max / sum and its own accumulator O_g = sum P_g V_g in TMEM;
-    // the halves are combined once per work item.  Thread t owns query row t (TMEM lane t).
-    const int g = (warp - 2) >> 2;  // warps 2-5: key half 0, warps 6-9: key half 1
+    const int s = (warp - 4) >> 2;         // warps 4-7: stream 0, warps 8-11: stream 1
     const int t = (warp & 3) * 32 + lane;  // a warp may only touch TMEM lanes 32 (warp % 4) .. + 31
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t o_own = lane_base + TM_O + 128 * g;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16) + TM_STREAM * s;
+    const uint32_t s_own = lane_base, o_own = lane_base + TM_OOFF;
     __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(p.ws + p.lay.op));
     const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
-    uint32_t s_count = 0, pv_waits = 0, items_done = 0;
+    uint32_t s_count = 0, items_done = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+    for (int item = N_STREAMS * blockIdx.x + s; item < p.n_items && ok; item += stride) {
       ItemInfo it;
       if (!load_item(p, item, it)) continue;
       const ClassStatic& cs = class_of(p, it.cls);
@@ -444,53 +511,55 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       rc.excl = reinterpret_cast<const uint32_t*>(p.ws + cs.excl_bits_off);
       rc.blk = reinterpret_cast<const uint32_t*>(p.ws + cs.blk_bits_off);
       rc.xpos = reinterpret_cast<const int32_t*>(p.ws + cs.x_pos_off);
-      const size_t orow = ((size_t)it.head * p.LP + it.qrow0 + r) * D + 64 * g;
+      const size_t orow = ((size_t)it.head * p.LP + it.qrow0 + r) * D;
 
       if (it.ntiles == 0) {
         if (rc.valid) {
           uint4* dst = reinterpret_cast<uint4*>(op + orow);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-          if (p.lse && g == 0) p.lse[(size_t)it.head * p.L + rc.qpos] = -INFINITY;
+          for (int i = 0; i < 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+          if (p.lse) p.lse[(size_t)it.head * p.L + rc.qpos] = -INFINITY;
         }
         continue;
       }
 
       float m_used = -INFINITY, l = 0.f;
-      uint32_t mk[2];
-      MaskRaw raw;
-      mask_prefetch(rc, __ldg(tiles + it.tile0), g, raw);
-      mask_finish(rc, raw, g, mk);
+      uint32_t tile = __ldg(tiles + it.tile0);
       for (int tt = 0; tt < it.ntiles; ++tt) {
-        const bool has_next = tt + 1 < it.ntiles;
-        if (has_next) mask_prefetch(rc, __ldg(tiles + it.tile0 + tt + 1), g, raw);
-
-        const uint32_t sb = s_count & 1, su = s_count >> 1;
-        if (!mbar_wait(&sm.s_full[sb], su & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        float s[64];
-        {
-          const uint32_t scol = lane_base + (sb ? TM_S1 : TM_S0) + 64 * g;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t rr[32];
-            tmem_ld32(scol + 32 * c, rr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[32 * c + j] = __uint_as_float(rr[j]);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&sm.s_free[sb]);
+        // tiles flagged full need no element mask (the flag is the same for the whole warp)
+        const bool full = (tile & TILE_FULL) != 0u;
+        MaskRaw raw;
+        if (!full) mask_prefetch(rc, tile, raw);  // the bitmap loads overlap the wait for S
+        if (tt + 1 < it.ntiles) tile = __ldg(tiles + it.tile0 + tt + 1);
+        if (!mbar_wait(&sm.s_full[s], s_count & 1, abort)) { ok = false; break; }
         ++s_count;
-
+        tc_fence_after();
+        float sv[128];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = ((mk[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(s_own + 32 * c, rr);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sv[32 * c + j] = __uint_as_float(rr[j]);
+        }
+        if (!full) {
+          uint32_t mk[4];
+          mask_finish(rc, raw, mk);
+          tmem_wait_ld();
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            if (__all_sync(0xFFFFFFFFu, mk[w] == 0xFFFFFFFFu)) continue;  // word open for the whole warp
+#pragma unroll
+            for (int c = 32 * w; c < 32 * w + 32; ++c) sv[c] = ((mk[w] >> (c & 31)) & 1u) ? sv[c] : -INFINITY;
+          }
+        } else {
+          tmem_wait_ld();
+        }
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
+        for (int c = 0; c < 128; c += 8) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], s[c + 2 * q], s[c + 2 * q + 1]);
+          for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], sv[c + 2 * q], sv[c + 2 * q + 1]);
         }
         const float mxs = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * p.scale_log2;
         float alpha = 1.f;
@@ -500,79 +569,57 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           m_used = mxs;
           resc = true;
         }
-
-        // the previous P_g V_g must be complete before P_g is overwritten or O_g rescaled
-        if (tt > 0) {
-          if (!mbar_wait(&sm.pv_done[g], pv_waits & 1, abort)) { ok = false; break; }
-          ++pv_waits;
-          tc_fence_after();
-          if (__any_sync(0xFFFFFFFFu, resc)) {
-            const float f = resc ? alpha : 1.f;
+        // S_s(tt) complete implies the previous P V of this stream is complete (same issuer,
+        // issue order), so O_s may be rescaled here
+        if (tt > 0 && __any_sync(0xFFFFFFFFu, resc)) {
+          const float f = resc ? alpha : 1.f;
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {  // 16 columns at a time: S stays live in registers
-              uint32_t oo[16];
-              tmem_ld16(o_own + 16 * c, oo);
-              tmem_wait_ld();
+          for (int c = 0; c < 8; ++c) {  // 16 columns at a time: S stays live in registers
+            uint32_t oo[16];
+            tmem_ld16(o_own + 16 * c, oo);
+            tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 16; ++j) oo[j] = __float_as_uint(__uint_as_float(oo[j]) * f);
-              tmem_st16(o_own + 16 * c, oo);
-            }
-            tmem_wait_st();
+            for (int j = 0; j < 16; ++j) oo[j] = __float_as_uint(__uint_as_float(oo[j]) * f);
+            tmem_st16(o_own + 16 * c, oo);
           }
         }
         const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-        // P row t, K-major 128B swizzle: atom g holds keys 64g..64g+63; chunk j -> j ^ (t & 7)
-        uint8_t* prow = sm.p + g * ATOM_BYTES + t * 128;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nb2 = make_float2(nb, nb);
+        float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // P row t over S columns [0, 64): column c holds keys 2c (low half) and 2c + 1.
+        // Exponent arguments and the row sum use the packed two-lane fp32 FMA / add.
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 4; ++h) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float a = ex2(fmaf(s[32 * h + 2 * c], p.scale_log2, nb));
-            const float b = ex2(fmaf(s[32 * h + 2 * c + 1], p.scale_log2, nb));
-            rs4[c & 3] += a + b;
-            pk[c] = pack_bf16x2(a, b);
+            const float2 x = __ffma2_rn(make_float2(sv[32 * h + 2 * c], sv[32 * h + 2 * c + 1]), sc2, nb2);
+            const float2 e = make_float2(ex2(x.x), ex2(x.y));
+            rs2[c & 1] = __fadd2_rn(rs2[c & 1], e);
+            pk[c] = pack_bf16x2(e.x, e.y);
           }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 v = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            *reinterpret_cast<uint4*>(prow + (((4 * h + j) ^ (t & 7)) << 4)) = v;
-          }
+          tmem_st16(s_own + 16 * h, pk);
         }
-        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
-        fence_proxy_async_smem();
+        l = l * alpha + ((rs2[0].x + rs2[1].x) + (rs2[0].y + rs2[1].y));
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sm.p_full[g]);
-        if (has_next) mask_finish(rc, raw, g, mk);
+        mbar_arrive(&sm.p_full[s]);
       }
       if (!ok) break;
-      // epilogue: both halves' last P V done, then O = (c0 O_0 + c1 O_1) / (c0 l0 + c1 l1)
-      if (!mbar_wait(&sm.pv_done[g], pv_waits & 1, abort)) { ok = false; break; }
-      ++pv_waits;
-      sm.xm[g][t] = m_used;
-      sm.xl[g][t] = l;
-      tc_fence_before();
-      named_bar_sync(1, 256);
+      // epilogue: the item's last P V done, then O = O_s / l
+      if (!mbar_wait(&sm.o_full[s], items_done & 1, abort)) { ok = false; break; }
+      ++items_done;
       tc_fence_after();
-      const float m0 = sm.xm[0][t], m1 = sm.xm[1][t];
-      const float M = fmaxf(m0, m1);
-      const float c0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M);
-      const float c1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
-      const float ltot = c0 * sm.xl[0][t] + c1 * sm.xl[1][t];
-      named_bar_sync(1, 256);  // both halves read before the next item's values land
-      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-      const float f0 = c0 * inv, f1 = c1 * inv;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
       uint4* dst = reinterpret_cast<uint4*>(op + orow);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t oa[32], ob[32];
-        tmem_ld32(lane_base + TM_O + 64 * g + 32 * c, oa);
-        tmem_ld32(lane_base + TM_O + 128 + 64 * g + 32 * c, ob);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t oa[32];
+        tmem_ld32(o_own + 32 * c, oa);
         tmem_wait_ld();
-        if (c == 1) {
+        if (c == 3) {
           tc_fence_before();
-          mbar_arrive(&sm.o_free);
+          mbar_arrive(&sm.o_free[s]);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -580,15 +627,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int k = 8 * j + 2 * e;
-            w[e] = pack_bf16x2(__uint_as_float(oa[k]) * f0 + __uint_as_float(ob[k]) * f1,
-                               __uint_as_float(oa[k + 1]) * f0 + __uint_as_float(ob[k + 1]) * f1);
+            w[e] = pack_bf16x2(__uint_as_float(oa[k]) * inv, __uint_as_float(oa[k + 1]) * inv);
           }
           if (rc.valid) dst[4 * c + j] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      ++items_done;
-      if (rc.valid && p.lse && g == 0)
-        p.lse[(size_t)it.head * p.L + rc.qpos] = (ltot > 0.f) ? (M + __log2f(ltot)) * 0.6931471805599453f : -INFINITY;
+      if (rc.valid && p.lse)
+        p.lse[(size_t)it.head * p.L + rc.qpos] = (l > 0.f) ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
   }
 
@@ -668,7 +713,7 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int grid = std::max(1, std::min(dp.n_items, sm_count()));
+  const int grid = std::max(1, std::min((dp.n_items + N_STREAMS - 1) / N_STREAMS, sm_count()));
   count_launches(1);
   msa_attn_kernel<<<grid, ATT_THREADS, smem, st>>>(mq, mqp, mk, mv, mk2, mv2, mxk, mxv, p);
   return cudaGetLastError();

@@ -586,6 +586,44 @@ __global__ void __launch_bounds__(TB_WARPS * 32) tiles_kernel(DevPlan dp, int bm
       }
       ntiles[item] = nt;
     }
+    nt = __shfl_sync(0xFFFFFFFFu, min(nt, cs.tile_cap), 0);
+    __syncwarp();
+    // ---- tiles that every row of the item attends to in full (sufficient conditions only)
+    const int32_t qpos_min = pos_of(row0);
+    for (int i = lane; i < nt; i += 32) {
+      const uint32_t t = out[i];
+      const int src = (int)(t >> 28);
+      const int32_t krow = (int32_t)(t & TILE_ROW_MASK);
+      bool full;
+      if (src == SRC_X) {  // gathered keys ascend by position; padding is never causal
+        full = at<const int32_t>(dp, cs.x_pos_off)[krow - cs.x_row0 + TILE - 1] <= qpos_min;
+      } else {
+        const int64_t kc0 = (int64_t)cs.kc_lo + (krow - cs.krow_lo), kc1 = kc0 + TILE - 1;
+        full = kc1 <= qc_min && kc1 < cs.kc_hi;  // causal for the first row, inside the region
+        if (full && !(cs.flags & CF_DENSE)) {
+          bool cover = ((cs.flags & CF_SINK) && kc1 < cs.sink) ||
+                       ((cs.flags & CF_BAND) && kc0 >= (int64_t)qc_max - cs.band + 1);
+          if (!cover && (cs.flags & CF_BLOCK)) {
+            const uint32_t* bits = at<const uint32_t>(dp, cs.blk_bits_off);
+            cover = true;
+            for (int qb = qc_min >> 6; qb <= (qc_max >> 6) && cover; ++qb)
+              for (int64_t kb = kc0 >> 6; kb <= (kc1 >> 6) && cover; ++kb)
+                cover = (bits[(size_t)qb * cs.blk_wpr + (kb >> 5)] >> (kb & 31)) & 1u;
+          }
+          full = cover;
+        }
+        if (full && (cs.flags & CF_EXCL)) {
+          const uint32_t* ex = at<const uint32_t>(dp, cs.excl_bits_off);
+          for (int64_t w = kc0 >> 5; w <= (kc1 >> 5) && full; ++w) {
+            const int lo = (w << 5) < kc0 ? (int)(kc0 - (w << 5)) : 0;
+            const int hi = ((w << 5) + 31) > kc1 ? (int)(kc1 - (w << 5)) : 31;
+            const uint32_t m = (hi - lo == 31) ? 0xFFFFFFFFu : (((1u << (hi - lo + 1)) - 1u) << lo);
+            full = (ex[w] & m) == 0u;
+          }
+        }
+      }
+      if (full) out[i] = t | TILE_FULL;
+    }
     __syncwarp();
   }
 }

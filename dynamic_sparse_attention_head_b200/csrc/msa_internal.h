@@ -15,6 +15,10 @@ constexpr int BLK = 64;         // block-sparse block
 constexpr int GRID_BAND = 64;   // default local band of grid heads
 constexpr int MAX_CLASSES_PER_HEAD = 2;
 constexpr int32_t POS_PAD = 0x7fffffff;  // position of a padding key (never causal)
+// Executed-tile id: source in bits 28-31, first key row in bits 0-26, and bit 27 set when every
+// row of the work item attends to all 128 keys of the tile (no element mask needed).
+constexpr uint32_t TILE_FULL = 1u << 27;
+constexpr uint32_t TILE_ROW_MASK = TILE_FULL - 1u;
 
 // key sources of a tile
 enum : int32_t { SRC_K = 0, SRC_K2D = 1, SRC_X = 2 };
@@ -135,7 +139,7 @@ struct Layout {
   int64_t segs;              // int32 [n_segments][3] start, len, modality
   int64_t class_dyn;         // ClassDyn [n_classes]
   int64_t item_ntiles;       // int32 [n_items]
-  int64_t tiles;             // uint32 [total tile capacity]: (src << 28) | first key row
+  int64_t tiles;             // uint32 [total tile capacity]: (src << 28) | TILE_FULL? | first key row
   int64_t modality;          // uint8 [L]
   int64_t rank;              // int32 [L]
   int64_t perm2d;            // int32 [L] modality-grouped order (text then video) -> position

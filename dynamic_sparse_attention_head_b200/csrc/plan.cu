@@ -909,8 +909,8 @@ msa_status msa_read_tiles(const msa_plan* P, const void* ws, int32_t head, int32
     rec.push_back(nt);
     for (int32_t k = 0; k < nt; ++k) {
       const int src = (int)(tl[k] >> 28);
-      const int32_t row = (int32_t)(tl[k] & 0x0FFFFFFFu);
-      rec.push_back(src);
+      const int32_t row = (int32_t)(tl[k] & TILE_ROW_MASK);
+      rec.push_back(src | ((tl[k] & TILE_FULL) ? 8 : 0));
       for (int cc = 0; cc < TILE; ++cc) {
         int32_t pos = -1;
         if (src == SRC_X) {

@@ -193,7 +193,8 @@ msa_status msa_tile_stats(const msa_plan* plan, const void* ws, int64_t tiles[2]
 
 /* Dumps the work list of head `head` for tests: for each of its 128-query work items the
  * query positions covered (-1 for padding) and, for every executed tile, its key source
- * (0 = keys in original order, 1 = modality-grouped keys, 2 = gathered keys) and the original
+ * (0 = keys in original order, 1 = modality-grouped keys, 2 = gathered keys; plus 8 when every
+ * query of the item attends to all 128 keys, so that the kernel applies no mask) and the original
  * positions of its 128 keys (-1 where a column holds no key, or a key the tile's mask leaves
  * to a gathered tile).  Flat int32 record:
  *   n_items, then per item: class, n_rows, rows[128], n_tiles, n_tiles x (src, keys[128]).

@@ -69,15 +69,21 @@ def test_tiles_cover_mask_exactly_once(name):
         mask = oracle.mask_rows(p, h, idx[h], np.arange(p.L)).astype(bool)
         cover = np.zeros((p.L, p.L), np.int32)
         seen_rows = np.zeros(p.L, np.int32)
+        n_full = 0
         for it in plan.read_tiles(h, ws):
             rows = it["rows"][it["rows"] >= 0]
             seen_rows[rows] += 1
-            for _, keys in it["tiles"]:
+            for _, keys, full in it["tiles"]:
                 kk = keys[keys >= 0]
                 cover[np.ix_(rows, kk)] += 1
+                if full:  # the kernel skips the element mask: every pair must be allowed
+                    assert len(kk) == 128 and mask[np.ix_(rows, kk)].all(), f"{name} head {h}: tile flagged full"
+                    n_full += 1
         assert np.all(seen_rows == 1), f"{name} head {h}: every query in exactly one work item"
         assert np.all(cover[mask] == 1), f"{name} head {h}: allowed pairs not covered exactly once"
         assert cover.max() <= 1, f"{name} head {h}: a key appears twice in one row's tiles"
+        if name == "ashape" and h == 0:  # local 256: tiles inside the band below the diagonal need no mask
+            assert n_full > 0, f"{name} head {h}: no tile flagged full"
 
 
 def test_dense_executes_causal_tiles_only():
@@ -89,3 +95,7 @@ def test_dense_executes_causal_tiles_only():
     # causal 128x128 tiles, the diagonal one split into two 64-key units when the row tile is ragged
     per_head = sum(((min(p.L, 128 * (i + 1)) - 1) // 64 + 2) // 2 for i in range(nq))
     assert tiles == p.Hq * per_head and items == p.Hq * nq
+    # every tile strictly below the diagonal of its 128-query item is flagged full
+    for h in range(p.Hq):
+        n_full = sum(full for it in plan.read_tiles(h, ws) for _, _, full in it["tiles"])
+        assert n_full == nq * (nq - 1) // 2
