@@ -52,6 +52,16 @@ constexpr int N_STREAMS = 2;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // one 128x128 bf16 tile
 constexpr uint32_t ATOM_BYTES = 128 * 128;      // one [128 rows][64 cols] 128B-swizzled atom
 
+// Per-row state of the element mask.
+struct RowCtx {
+  int valid, qpos, qcoord;
+  int flags, sink, band, kc_lo, kc_hi, krow_lo, x_row0, nwords, blk_wpr;
+  const uint32_t* slash;
+  const uint32_t* excl;
+  const uint32_t* blk;
+  const int32_t* xpos;
+};
+
 struct __align__(1024) AttnSmem {
   uint8_t q[N_STREAMS][TILE_BYTES];
   uint8_t k[N_STREAMS][TILE_BYTES];
@@ -62,6 +72,7 @@ struct __align__(1024) AttnSmem {
   uint64_t s_full[N_STREAMS], p_full[N_STREAMS];
   uint64_t o_full[N_STREAMS], o_free[N_STREAMS];
   uint64_t drain[N_STREAMS];
+  RowCtx rctx[256];  // mask state of the row of each softmax thread (read off the critical path)
   uint32_t tmem_base;
   int abort;
   int issue_lock;
@@ -115,15 +126,6 @@ __device__ __forceinline__ bool next_work(const AttnParams& p, int& item, int st
   return false;
 }
 
-// Per-row state of the element mask.
-struct RowCtx {
-  int valid, qpos, qcoord;
-  int flags, sink, band, kc_lo, kc_hi, krow_lo, x_row0, nwords, blk_wpr;
-  const uint32_t* slash;
-  const uint32_t* excl;
-  const uint32_t* blk;
-  const int32_t* xpos;
-};
 
 // Bits [0, n) of the 32-column word w of a 128-column row (n clipped to [0, 128]).
 __device__ __forceinline__ uint32_t low_bits(int n, int w) {
@@ -493,7 +495,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       if (!load_item(p, item, it)) continue;
       const ClassStatic& cs = class_of(p, it.cls);
       const int r = it.row0 + t;
-      RowCtx rc;
+      RowCtx& rc = sm.rctx[threadIdx.x - 128];
       rc.valid = r < it.nrows;
       const int32_t* rows = reinterpret_cast<const int32_t*>(p.ws + cs.rows_off);
       rc.qpos = rc.valid ? ((cs.flags & CF_PERMUTED) ? __ldg(rows + r) : r) : 0;
@@ -524,13 +526,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
 
       float m_used = -INFINITY, l = 0.f;
-      uint32_t tile = __ldg(tiles + it.tile0);
+      // The element mask of a tile is built before its S is waited for (for the first tile
+      // here, for the others right after the previous tile's P is handed over), so that the
+      // bitmap loads and the bit arithmetic overlap the tensor core's work.  Tiles flagged full
+      // need no mask (the flag is the same for the whole warp).
+      uint32_t mk[4];
+      bool full;
+      auto build_mask = [&](uint32_t t) {
+        full = (t & TILE_FULL) != 0u;
+        if (!full) {
+          MaskRaw raw;
+          mask_prefetch(rc, t, raw);
+          mask_finish(rc, raw, mk);
+        }
+      };
+      build_mask(__ldg(tiles + it.tile0));
       for (int tt = 0; tt < it.ntiles; ++tt) {
-        // tiles flagged full need no element mask (the flag is the same for the whole warp)
-        const bool full = (tile & TILE_FULL) != 0u;
-        MaskRaw raw;
-        if (!full) mask_prefetch(rc, tile, raw);  // the bitmap loads overlap the wait for S
-        if (tt + 1 < it.ntiles) tile = __ldg(tiles + it.tile0 + tt + 1);
+        const uint32_t tile_next = (tt + 1 < it.ntiles) ? __ldg(tiles + it.tile0 + tt + 1) : 0u;
         if (!mbar_wait(&sm.s_full[s], s_count & 1, abort)) { ok = false; break; }
         ++s_count;
         tc_fence_after();
@@ -543,8 +555,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           for (int j = 0; j < 32; ++j) sv[32 * c + j] = __uint_as_float(rr[j]);
         }
         if (!full) {
-          uint32_t mk[4];
-          mask_finish(rc, raw, mk);
           tmem_wait_ld();
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
@@ -604,6 +614,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[s]);
+        if (tt + 1 < it.ntiles) build_mask(tile_next);
       }
       if (!ok) break;
       // epilogue: the item's last P V done, then O = O_s / l
