@@ -281,9 +281,11 @@ __global__ void __launch_bounds__(LQ_THREADS) lastq_pass2(DevPlan dp, const __nv
   const int64_t c0 = std::max<int64_t>(0, own0 - span64);
   const int nblk = (int)((own1 - c0 + KB - 1) / KB);
   int32_t min_rc = 0x7fffffff, max_rc = -0x7fffffff;
+  bool contig = true;  // row coordinates rcs[r] = rcs[0] + r: each offset is one diagonal of a block
   for (int r = 0; r < rs.n_rows; ++r) {
     min_rc = min(min_rc, rs.rcs[r]);
     max_rc = max(max_rc, rs.rcs[r]);
+    contig = contig && rs.rcs[r] == rs.rcs[0] + r;
   }
   const int64_t obase = (int64_t)min_rc - (own0 + rs.chunk - 1);
   const int64_t ocount = (int64_t)max_rc - c0 - obase + 1;
@@ -334,7 +336,29 @@ __global__ void __launch_bounds__(LQ_THREADS) lastq_pass2(DevPlan dp, const __nv
       }
     }
     // slash sums: offsets touched by this block, rows in order
-    if (slash) {
+    if (slash && contig) {
+      // offset o = rcs[0] + d - j0 collects the elements (r, r - d) of diagonal d; one thread
+      // per diagonal, rows ascending (the order of the general loop below)
+      const bool inside = j0 >= rs.slash_lo && j0 + KB <= rs.slash_hi;
+      const int n_rows = rs.n_rows;
+      for (int dd = threadIdx.x; dd < n_rows + KB - 1; dd += LQ_THREADS) {
+        const int d = dd - (KB - 1);
+        const int64_t si = (int64_t)min_rc + d - j0 - obase;
+        if (si < 0 || si >= SACC_MAX) continue;
+        const int r_lo = max(0, d), r_hi = min(n_rows, KB + d);
+        float acc = 0.f;
+        if (inside) {
+          for (int r = r_lo; r < r_hi; ++r) acc += sm.a[r * (KB + 1) + (r - d)];
+        } else {
+          for (int r = r_lo; r < r_hi; ++r) {
+            const int64_t j = j0 + (r - d);
+            if (j < rs.slash_lo || j >= rs.slash_hi) continue;
+            acc += sm.a[r * (KB + 1) + (r - d)];
+          }
+        }
+        sacc[si] += acc;
+      }
+    } else if (slash) {
       const int64_t olo = (int64_t)min_rc - (j0 + KB - 1), ohi = (int64_t)max_rc - j0;
       for (int64_t o = olo + threadIdx.x; o <= ohi; o += LQ_THREADS) {
         const int64_t si = o - obase;
