@@ -55,7 +55,7 @@ __global__ void group_rows_kernel(DevPlan dp, const __nv_bfloat16* src, int64_t 
 constexpr int LQ_THREADS = 128;
 constexpr int KB = 64;       // keys per block
 constexpr int PAD = 136;     // bf16 row pitch in shared memory (272 bytes: conflict-free fragments)
-constexpr int SACC_MAX = 1024 + 2 * 4096 + 128;
+constexpr int SACC_MAX = 4096 + 1024 + 4096 + 64;  // largest accumulator: span 4096, chunk 1024
 
 struct LqSmem {
   __nv_bfloat16 q[LASTQ * PAD];
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(LQ_THREADS) lastq_pass2(DevPlan dp, const __nv
   const int64_t obase = (int64_t)min_rc - (own0 + rs.chunk - 1);
   const int64_t ocount = (int64_t)max_rc - c0 - obase + 1;
   if (slash)
-    for (int64_t i = threadIdx.x; i < ocount && i < SACC_MAX; i += LQ_THREADS) sacc[i] = 0.f;
+    for (int64_t i = threadIdx.x; i < ocount && i < dp.sacc_n; i += LQ_THREADS) sacc[i] = 0.f;
   load_kblock(sm, 0, ks, c0, own1);
   cp_async_commit();
   __syncthreads();
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(LQ_THREADS) lastq_pass2(DevPlan dp, const __nv
       for (int dd = threadIdx.x; dd < n_rows + KB - 1; dd += LQ_THREADS) {
         const int d = dd - (KB - 1);
         const int64_t si = (int64_t)min_rc + d - j0 - obase;
-        if (si < 0 || si >= SACC_MAX) continue;
+        if (si < 0 || si >= dp.sacc_n) continue;
         const int r_lo = max(0, d), r_hi = min(n_rows, KB + d);
         float acc = 0.f;
         if (inside) {
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(LQ_THREADS) lastq_pass2(DevPlan dp, const __nv
       const int64_t olo = (int64_t)min_rc - (j0 + KB - 1), ohi = (int64_t)max_rc - j0;
       for (int64_t o = olo + threadIdx.x; o <= ohi; o += LQ_THREADS) {
         const int64_t si = o - obase;
-        if (si < 0 || si >= SACC_MAX) continue;
+        if (si < 0 || si >= dp.sacc_n) continue;
         float s = 0.f;
         for (int r = 0; r < rs.n_rows; ++r) {
           const int64_t cc = (int64_t)sm.rcs[r] - o - j0;
@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(LQ_THREADS) lastq_pass2(DevPlan dp, const __nv
       const int64_t o = (int64_t)max_rc - j;
       if (o < 0 || o >= dp.L) continue;
       const int64_t si = o - obase;
-      sout[o] = (si >= 0 && si < SACC_MAX) ? sacc[si] : 0.f;
+      sout[o] = (si >= 0 && si < dp.sacc_n) ? sacc[si] : 0.f;
     }
   }
 }
@@ -593,6 +593,8 @@ cudaError_t launch_lastq(const DevPlan& dp, const void* Q, const void* K, const 
     cudaFuncSetAttribute(lastq_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
     configured = true;
   }
+  if (dp.sacc_n < 0 || dp.sacc_n > SACC_MAX) return cudaErrorInvalidValue;
+  const size_t smem2_used = sizeof(LqSmem) + sizeof(float) * (size_t)dp.sacc_n;
   const dim3 grid(dp.max_chunks, dp.n_rowsets);
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
   count_launches(3);
@@ -600,7 +602,7 @@ cudaError_t launch_lastq(const DevPlan& dp, const void* Q, const void* K, const 
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   lastq_combine<<<dp.n_rowsets, LASTQ, 0, st>>>(dp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  lastq_pass2<<<grid, LQ_THREADS, smem2, st>>>(dp, q, s.q_head, s.q_row, K, s.k_head, s.k_row);
+  lastq_pass2<<<grid, LQ_THREADS, smem2_used, st>>>(dp, q, s.q_head, s.q_row, K, s.k_head, s.k_row);
   return cudaGetLastError();
 }
 

@@ -21,6 +21,7 @@ struct DevPlan {
   int64_t n_text;      // text tokens (they lead the modality-grouped order)
   int32_t tb_words;    // unit-bitmap words per tile-builder warp
   int32_t max_chunks;  // most key chunks of any row set
+  int32_t sacc_n;      // slash accumulator entries the second estimation pass needs per block
   float scale;
   const int32_t* class_kind;  // host copy: kind of each class
 };

@@ -170,6 +170,7 @@ extern "C" msa_status msa_vslash_estimate_static(const void* Q, const void* K, i
   dp.n_rowsets = 1;
   dp.n_jobs = 2;
   dp.max_chunks = n_chunks;
+  dp.sacc_n = (LASTQ - 1) + (int32_t)NOALLOC_CHUNK + 64 + 64;  // consecutive rows: span 63
   dp.scale = scale;
   dp.has2d = 0;
   msa_strides s{};

@@ -372,13 +372,29 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
       default: break;
     }
   }
+  // Key chunks of the estimation passes (one block each): 1024 keys, halved down to 256 while
+  // the passes would launch fewer than eight blocks per SM.
+  int32_t chunk = 1024;
+  {
+    int64_t blocks = 0;
+    for (const auto& r : RS) blocks += (r.key_hi + chunk - 1) / chunk;
+    while (chunk > 256 && blocks < 8LL * sm_count()) {
+      chunk /= 2;
+      blocks = 0;
+      for (const auto& r : RS) blocks += (r.key_hi + chunk - 1) / chunk;
+    }
+  }
+  int32_t sacc_n = 0;
   for (auto& r : RS) {
     if (r.span > 4096) {
       delete P;
       return MSA_ERR_UNSUPPORTED;
     }
-    r.chunk = 1024;
+    r.chunk = chunk;
     r.n_chunks = (int32_t)((r.key_hi + r.chunk - 1) / r.chunk);
+    // offsets one block of pass 2 touches: the rows' spread, its chunk and the look-back
+    const int32_t span64 = (r.span + 63) / 64 * 64;
+    sacc_n = std::max(sacc_n, r.span + chunk + span64 + 64);
   }
 
   // ---- layout
@@ -566,6 +582,7 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   for (const auto& r : RS) mc = std::max(mc, r.n_chunks);
   dp.tb_words = tbw;
   dp.max_chunks = mc;
+  dp.sacc_n = sacc_n;
   dp.class_kind = P->class_kind.data();
   *out = P;
   return MSA_OK;
