@@ -3,8 +3,9 @@
 // MMInference ("key machinery"): block-sparse FlashAttention-style kernels load only the
 // permuted blocks and keep the tensor-core compute dense; "Grid-Shape Flash Attention"
 // (Algorithm 5) is the FlashAttention-2 online softmax over those blocks.  Here:
-//  - one persistent CTA per SM runs two independent streams of 128-query work items
-//    (stream s takes items 2 b + s, 2 b + s + 2 G, ... of CTA b in a grid of G);
+//  - one persistent CTA per SM runs two independent streams of 128-query work items; each
+//    stream takes the next item from a global counter when it needs one (items are in
+//    plan order, most keys first, so the greedy assignment balances the SMs);
 //  - warps 0 and 2 stream the Q, K and V tiles of stream 0 and 1 with TMA (128-byte
 //    swizzle) into single-buffered slots of their own;
 //  - warps 1 and 3 (one thread each) issue the tcgen05.mma of stream 0 and 1:
@@ -39,6 +40,7 @@ struct AttnParams {
   int32_t n_items;
   float scale_log2;        // softmax scale * log2(e)
   float* lse;              // [Hq][L] or null
+  uint32_t* next_item;     // work-item counter, zero at launch
 };
 
 // warpgroup 0: warps 0 / 2 TMA of stream 0 / 1, warps 1 / 3 MMA of stream 0 / 1; warpgroups
@@ -49,6 +51,9 @@ constexpr int ATT_THREADS = 384;
 constexpr int REG_CTRL = 72, REG_SOFTMAX = 216;
 static_assert(128 * REG_CTRL + 256 * REG_SOFTMAX <= ATT_THREADS * 168, "register split exceeds the launch allocation");
 constexpr int N_STREAMS = 2;
+constexpr int IQ_DEPTH = 4;
+// readers of a queue entry: the MMA issuer, the V loads of the TMA thread, 128 softmax threads
+constexpr uint32_t IQ_READERS = 130;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // one 128x128 bf16 tile
 constexpr uint32_t ATOM_BYTES = 128 * 128;      // one [128 rows][64 cols] 128B-swizzled atom
 
@@ -71,6 +76,10 @@ struct __align__(1024) AttnSmem {
   uint64_t v_full[N_STREAMS], v_empty[N_STREAMS];
   uint64_t s_full[N_STREAMS], p_full[N_STREAMS];
   uint64_t o_full[N_STREAMS], o_free[N_STREAMS];
+  // work-item queue of each stream: ids taken from the global counter by the stream's TMA
+  // thread, read by its MMA issuer and softmax warpgroup (-1 ends the stream)
+  int32_t iq[N_STREAMS][IQ_DEPTH];
+  uint64_t iq_full[N_STREAMS][IQ_DEPTH], iq_empty[N_STREAMS][IQ_DEPTH];
   uint64_t drain[N_STREAMS];
   RowCtx rctx[256];  // mask state of the row of each softmax thread (read off the critical path)
   uint32_t tmem_base;
@@ -117,13 +126,6 @@ __device__ __forceinline__ bool load_item(const AttnParams& p, int item, ItemInf
   it.x_slice = (int)hs.x_slice;
   if (it.row0 >= it.nrows) it.ntiles = -1;  // no rows: item skipped by every role
   return it.ntiles >= 0;
-}
-
-// Advances `item` (in steps of `stride`) to the next item with at least one tile.
-__device__ __forceinline__ bool next_work(const AttnParams& p, int& item, int stride, ItemInfo& it) {
-  for (; item < p.n_items; item += stride)
-    if (load_item(p, item, it) && it.ntiles > 0) return true;
-  return false;
 }
 
 
@@ -301,7 +303,7 @@ __device__ __forceinline__ void issue_unlock(int* lock) { atomicExch(lock, 0); }
 // stream whose group follows the other's gets its S one group later and starts its softmax
 // then: the streams settle half a cycle apart, and one stream's MMAs run while the other
 // computes its softmax.
-__device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, uint32_t tmem, int s, int stride,
+__device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, uint32_t tmem, int s,
                                            volatile int* abort) {
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
@@ -323,8 +325,14 @@ __device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, ui
     if (last) umma_commit(&sm.q_empty[s]);
     ++k_use;
   };
-  ItemInfo it;
-  for (int item = N_STREAMS * blockIdx.x + s; next_work(p, item, stride, it); item += stride) {
+  for (uint32_t qi = 0;; ++qi) {
+    const uint32_t slot = qi % IQ_DEPTH;
+    if (!mbar_wait(&sm.iq_full[s][slot], (qi / IQ_DEPTH) & 1, abort)) return;
+    const int item = sm.iq[s][slot];
+    mbar_arrive(&sm.iq_empty[s][slot]);
+    if (item < 0) break;
+    ItemInfo it;
+    if (!load_item(p, item, it) || it.ntiles == 0) continue;
     const int n = it.ntiles;
     if (!mbar_wait(&sm.q_full[s], q_use & 1, abort)) return;
     ++q_use;
@@ -373,7 +381,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int lane = threadIdx.x & 31;
   volatile int* abort = &sm.abort;
   uint32_t* err = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.ws + p.lay.header));
-  const int stride = N_STREAMS * gridDim.x;
 
   if (threadIdx.x == 0) {
     sm.abort = 0;
@@ -390,6 +397,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&sm.o_full[s], 1);
       mbar_init(&sm.o_free[s], 128);
       mbar_init(&sm.drain[s], 1);
+      for (int i = 0; i < IQ_DEPTH; ++i) {
+        mbar_init(&sm.iq_full[s][i], 1);
+        mbar_init(&sm.iq_empty[s][i], IQ_READERS);
+      }
     }
     fence_barrier_init();
   }
@@ -412,14 +423,39 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
-      int qk_item = N_STREAMS * blockIdx.x + s, v_item = qk_item, qk_op = 0, v_j = 0;
+      // Work items come from the global counter in plan order (most keys first), one at a
+      // time into the stream's queue: the Q/K loads take them as they come, the V loads
+      // follow the same sequence from the queue.
+      uint32_t published = 0;
+      bool ended = false;
+      auto publish = [&]() -> bool {
+        const uint32_t slot = published % IQ_DEPTH, use = published / IQ_DEPTH;
+        if (ended || (use > 0 && !mbar_test(&sm.iq_empty[s][slot], (use - 1) & 1))) return false;
+        int id = (int)atomicAdd(p.next_item, 1u);
+        if (id >= p.n_items) id = -1;
+        ended = id < 0;
+        sm.iq[s][slot] = id;
+        mbar_arrive(&sm.iq_full[s][slot]);
+        ++published;
+        return true;
+      };
+      uint32_t qk_q = 0, v_q = 0;  // queue positions of the items the two load sequences are on
+      int qk_op = -1, v_j = -1;    // -1: no item yet
       ItemInfo qk_it, v_it;
-      bool qk_live = next_work(p, qk_item, stride, qk_it);
-      bool v_live = next_work(p, v_item, stride, v_it);
+      bool qk_live = true, v_live = true;
       uint32_t q_iss = 0, k_iss = 0, v_iss = 0;
       Watchdog wd;
       while (qk_live || v_live) {
-        if (qk_live) {
+        if (qk_live && qk_op < 0) {  // next item of the Q/K loads
+          if (published <= qk_q && publish()) wd.progress();
+          if (published > qk_q) {
+            const int id = sm.iq[s][qk_q % IQ_DEPTH];
+            if (id < 0) qk_live = false;
+            else if (!load_item(p, id, qk_it) || qk_it.ntiles == 0) ++qk_q;
+            else qk_op = 0;
+          }
+        }
+        if (qk_live && qk_op >= 0) {
           if (qk_op == 0) {
             if (q_iss == 0 || mbar_test(&sm.q_empty[s], (q_iss - 1) & 1)) {
               mbar_arrive_expect_tx(&sm.q_full[s], TILE_BYTES);
@@ -441,23 +477,35 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             ++k_iss;
             wd.progress();
             if (j + 1 == qk_it.ntiles) {
-              qk_item += stride;
-              qk_live = next_work(p, qk_item, stride, qk_it);
-              qk_op = 0;
+              ++qk_q;
+              qk_op = -1;
             } else {
               qk_op = j + 2;
             }
           }
         }
-        if (v_live && (v_iss == 0 || mbar_test(&sm.v_empty[s], (v_iss - 1) & 1))) {
+        if (v_live && v_j < 0 && published > v_q) {  // next item of the V loads
+          const uint32_t slot = v_q % IQ_DEPTH;
+          const int id = sm.iq[s][slot];
+          if (id < 0) {
+            mbar_arrive(&sm.iq_empty[s][slot]);
+            v_live = false;
+          } else if (!load_item(p, id, v_it) || v_it.ntiles == 0) {
+            mbar_arrive(&sm.iq_empty[s][slot]);
+            ++v_q;
+          } else {
+            v_j = 0;
+          }
+        }
+        if (v_live && v_j >= 0 && (v_iss == 0 || mbar_test(&sm.v_empty[s], (v_iss - 1) & 1))) {
           issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, true, __ldg(tiles + v_it.tile0 + v_j), v_it, sm.v[s],
                    &sm.v_full[s]);
           ++v_iss;
           wd.progress();
           if (++v_j == v_it.ntiles) {
-            v_item += stride;
-            v_live = next_work(p, v_item, stride, v_it);
-            v_j = 0;
+            mbar_arrive(&sm.iq_empty[s][v_q % IQ_DEPTH]);
+            ++v_q;
+            v_j = -1;
           }
         }
         if (wd.expired(abort)) {
@@ -473,7 +521,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // ------------------------------------------------------------------ MMA issuers
     // warp 1: stream 0, warp 3: stream 1
     if (lane == 0) {
-      mma_stream(p, sm, tmem, warp >> 1, stride, abort);
+      mma_stream(p, sm, tmem, warp >> 1, abort);
       // wait for every MMA issued by this thread before the tensor memory is released
       umma_commit(&sm.drain[warp >> 1]);
       mbar_wait(&sm.drain[warp >> 1], 0, abort, 100000000ull);
@@ -490,7 +538,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
     uint32_t s_count = 0, items_done = 0;
     bool ok = true;
-    for (int item = N_STREAMS * blockIdx.x + s; item < p.n_items && ok; item += stride) {
+    for (uint32_t qi = 0; ok; ++qi) {
+      const uint32_t slot = qi % IQ_DEPTH;
+      if (!mbar_wait(&sm.iq_full[s][slot], (qi / IQ_DEPTH) & 1, abort)) break;
+      const int item = sm.iq[s][slot];
+      mbar_arrive(&sm.iq_empty[s][slot]);
+      if (item < 0) break;
       ItemInfo it;
       if (!load_item(p, item, it)) continue;
       const ClassStatic& cs = class_of(p, it.cls);
@@ -717,6 +770,9 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
   p.n_items = dp.n_items;
   p.scale_log2 = dp.scale * 1.4426950408889634f;
   p.lse = lse;
+  // work items are handed out by a counter in the workspace header, zeroed here
+  p.next_item = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(ws + dp.lay.header)) + HDR_NEXT_ITEM;
+  if (cudaError_t e = cudaMemsetAsync(p.next_item, 0, sizeof(uint32_t), st)) return e;
   const size_t smem = sizeof(AttnSmem);
   static bool configured = false;
   if (!configured) {

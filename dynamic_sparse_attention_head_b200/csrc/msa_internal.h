@@ -18,6 +18,7 @@ constexpr int32_t POS_PAD = 0x7fffffff;  // position of a padding key (never cau
 // Executed-tile id: source in bits 28-31, first key row in bits 0-26, and bit 27 set when every
 // row of the work item attends to all 128 keys of the tile (no element mask needed).
 constexpr uint32_t TILE_FULL = 1u << 27;
+constexpr int HDR_NEXT_ITEM = 2;  // header word: next work item of the attention kernel
 constexpr uint32_t TILE_ROW_MASK = TILE_FULL - 1u;
 
 // key sources of a tile
@@ -130,7 +131,7 @@ struct WorkItem {
 
 // Byte offsets of the workspace regions.
 struct Layout {
-  int64_t header;            // uint32 [64]: [0] error bits, [1] ready flags, [8..] stats
+  int64_t header;            // uint32 [64]: [0] error bits, [1] ready flags, [2] attention work-item counter, [8..] stats
   int64_t classes;           // ClassStatic [n_classes]
   int64_t heads;             // HeadStatic [Hq]
   int64_t rowsets;           // RowSet [n_rowsets]
