@@ -347,25 +347,28 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_sweep(args):
-    """The budget sweep on the LLaMA-3-8B-shaped layer: one JSON line per (L, budget), with the
-    estimation time against the attention time.  Not the benchmark line: a table."""
+    """The budget sweep on the LLaMA-3-8B-shaped layer: one JSON line per (L, budget) with the
+    per-stage times, estimation against attention.  A table, not the benchmark line.  The
+    text-only layers' inputs depend on L alone, so they are generated once per length; layers
+    of 512K tokens and more are timed over fewer repetitions (1 warm-up, 2 timed)."""
     import torch
     import dynamic_sparse_attention_head_b200 as msa
     lengths = [int(x) for x in args.sweep_lengths.split(",")]
     budgets = [None if x == "dense" else float(x) for x in args.sweep_budgets.split(",")]
     for L in lengths:
+        warm, steps = (args.warmup, args.steps) if L <= 131072 else (1, 2)
+        Qh, Kh, Vh = make_host_inputs(workload.sweep_layer(L, None), seed=0)
+        q, k, v = (torch.from_numpy(x).view(torch.bfloat16).cuda() for x in (Qh, Kh, Vh))
+        del Qh, Kh, Vh
+        o = torch.empty_like(q)
         for b in budgets:
             p = workload.sweep_layer(L, b)
-            Qh, Kh, Vh = make_host_inputs(p, seed=0)
-            q, k, v = (torch.from_numpy(x).view(torch.bfloat16).cuda() for x in (Qh, Kh, Vh))
-            del Qh, Kh, Vh
-            o = torch.empty_like(q)
             plan = msa.Plan(p)
             ws = plan.alloc_workspace()
             st = torch.cuda.current_stream()
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
             stages = []
-            for i in range(args.warmup + args.steps):
+            for i in range(warm + steps):
                 ev[0].record(st)
                 plan.estimate(q, k, ws)
                 ev[1].record(st)
@@ -376,21 +379,24 @@ def run_sweep(args):
                 plan.unpermute(ws, o)
                 ev[4].record(st)
                 torch.cuda.synchronize()
-                if i >= args.warmup:
+                if i >= warm:
                     stages.append([ev[j].elapsed_time(ev[j + 1]) for j in range(4)])
             assert plan.device_status(ws) == 0
             tiles, _ = plan.tile_stats(ws)
             st_ms = np.mean(np.array(stages), axis=0)
             flops = msa.executed_flops(tiles)
-            print(json.dumps({"sweep": "llama3-8b-text", "L": L, "budget": b, "ms_per_layer": float(st_ms.sum()),
-                              "estimate_ms": float(st_ms[0]), "permute_ms": float(st_ms[1]),
-                              "attention_ms": float(st_ms[2]), "unpermute_ms": float(st_ms[3]),
+            print(json.dumps({"sweep": "llama3-8b-text", "L": L, "budget": b, "warmup": warm, "steps": steps,
+                              "ms_per_layer": float(st_ms.sum()), "estimate_ms": float(st_ms[0]),
+                              "permute_ms": float(st_ms[1]), "attention_ms": float(st_ms[2]),
+                              "unpermute_ms": float(st_ms[3]),
                               "estimate_over_attention": float(st_ms[0] / st_ms[2]),
                               "executed_flops": flops, "dense_causal_flops": dense_causal_flops(p),
                               "density": flops / dense_causal_flops(p),
                               "attn_tflops": flops / (st_ms[2] * 1e-3) / 1e12}), flush=True)
-            del q, k, v, o, ws, plan
+            del ws, plan
             torch.cuda.empty_cache()
+        del q, k, v, o
+        torch.cuda.empty_cache()
 
 
 def run_reference(args, rank, world):
