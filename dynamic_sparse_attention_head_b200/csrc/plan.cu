@@ -297,10 +297,12 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
     H.q_rows = perm ? LP : 0;
     x_rows_max = std::max(x_rows_max, xr);
   }
-  // ---- work items: grouped by KV head and, within a head, by key source (the items in flight
-  // then share one copy of one head's K and V, which stays in L2 while the group runs); within
-  // a group slots from the last (most keys) to the first with the query heads interleaved, so
-  // that the dynamic assignment in the attention kernel hands out the longest items first
+  // ---- work items: grouped by KV head, then key source, then head kind.  The items in flight
+  // then read one copy of one head's K and V (which stays in L2 while the group runs, where it
+  // fits) and move through it at about the same pace (items of one kind cost about the same per
+  // tile), so that they reuse each other's tiles in L2.  Within a group: slots from the last
+  // (most keys) to the first with the query heads interleaved, so that the dynamic assignment
+  // in the attention kernel hands out the longest items first.
   {
     int32_t max_slots = 0;
     for (auto& c : C) {
@@ -312,9 +314,11 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
     for (int c = 0; c < (int)C.size(); ++c) C[c].item0 = -1;
     for (int32_t g = 0; g < prob->Hkv; ++g)
       for (int32_t src : {SRC_K, SRC_K2D})  // K/V in original order, then the modality-grouped copy
-        for (int32_t s = max_slots - 1; s >= 0; --s)
-          for (int c = 0; c < (int)C.size(); ++c)
-            if (C[c].kvh == g && C[c].k_src == src && s < C[c].n_items) P->items.push_back(WorkItem{c, s});
+        for (int32_t kind = MSA_DENSE; kind <= MSA_BOUND2D; ++kind)
+          for (int32_t s = max_slots - 1; s >= 0; --s)
+            for (int c = 0; c < (int)C.size(); ++c)
+              if (C[c].kvh == g && C[c].k_src == src && prob->heads[C[c].head].kind == kind && s < C[c].n_items)
+                P->items.push_back(WorkItem{c, s});
     int64_t tb = 0;
     for (auto& c : C) {
       c.tile_base = tb;
