@@ -512,35 +512,85 @@ __global__ void __launch_bounds__(TK_THREADS) topk_jobs_kernel(DevPlan dp) {
 // block-sparse estimation
 // ---------------------------------------------------------------------------------------
 // mean of each 64-row block, fp32, rows summed in order
-__global__ void pool_kernel(DevPlan dp, const __nv_bfloat16* X, int64_t xh, int64_t xr, int n_heads, int q_side) {
-  const int h = blockIdx.y;
+// Mean of each 64-row block of K (grid rows y < Hkv: KV head y) and of Q (rows y >= Hkv: the
+// (y - Hkv)-th block-sparse query head), one launch for both.  One CTA of 256 threads per
+// block: 16 lanes cover a 256-byte row with 16-byte loads, 16 row groups take rows g, g + 16,
+// g + 32, g + 48, and the 16 partial sums of each column are added in row-group order.
+constexpr int POOL_THREADS = 256;
+__global__ void __launch_bounds__(POOL_THREADS) pool_kernel(DevPlan dp, const __nv_bfloat16* Q, int64_t qh,
+                                                            int64_t qr, const __nv_bfloat16* K, int64_t kh,
+                                                            int64_t kr) {
+  __shared__ float part[16][D + 4];
+  const bool q_side = (int)blockIdx.y >= dp.Hkv;
+  int h = blockIdx.y;
   if (q_side) {
-    const HeadStatic& hs = at<const HeadStatic>(dp, dp.lay.heads)[h];
-    if (hs.kind != MSA_BLOCK) return;
+    const HeadStatic* hs = at<const HeadStatic>(dp, dp.lay.heads);
+    int seen = -1;
+    for (h = 0; h < dp.Hq; ++h)
+      if (hs[h].kind == MSA_BLOCK && ++seen == (int)blockIdx.y - dp.Hkv) break;
+    if (h >= dp.Hq) return;
   }
   float* out = q_side ? at<float>(dp, at<const HeadStatic>(dp, dp.lay.heads)[h].qbar_off)
                       : at<float>(dp, dp.lay.kbar) + (int64_t)h * dp.nb * D;
-  const int d = threadIdx.x;
+  const __nv_bfloat16* X = q_side ? Q + (int64_t)h * qh : K + (int64_t)h * kh;
+  const int64_t xr = q_side ? qr : kr;
+  const int sub = threadIdx.x & 15, g = threadIdx.x >> 4;
+  auto load = [&](int b, uint4 (&v)[4]) {
+    const __nv_bfloat16* src = X + (int64_t)b * BLK * xr + sub * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)(g + 16 * i) * xr));
+  };
+  uint4 nxt[4];
+  if ((int)blockIdx.x < dp.nb) load(blockIdx.x, nxt);
   for (int b = blockIdx.x; b < dp.nb; b += gridDim.x) {
-    const __nv_bfloat16* src = X + (int64_t)h * xh + (int64_t)b * BLK * xr + d;
-    float s = 0.f;
-    for (int r = 0; r < BLK; ++r) s += __bfloat162float(src[(int64_t)r * xr]);
-    out[(int64_t)b * D + d] = s * (1.f / BLK);
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = nxt[i];
+    if (b + (int)gridDim.x < dp.nb) load(b + gridDim.x, nxt);  // next block's rows in flight meanwhile
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p2[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[g][sub * 8 + e] = acc[e];
+    __syncthreads();
+    if (threadIdx.x < D) {
+      float t = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) t += part[j][threadIdx.x];
+      out[(int64_t)b * D + threadIdx.x] = t * (1.f / BLK);
+    }
+    __syncthreads();
   }
-  (void)n_heads;
 }
 
 constexpr int BT_THREADS = 256;
 
-// one CTA per (query block, head): pooled logits of key blocks c <= b, then top-k
+// one CTA per (query block, block-sparse head): pooled logits of key blocks c <= b, then top-k
 __global__ void __launch_bounds__(BT_THREADS) block_topk_kernel(DevPlan dp) {
   extern __shared__ uint32_t bt_keys[];
   __shared__ uint32_t hist[258];
   __shared__ int scan_sh[32];
   __shared__ __align__(16) float qb[D];
-  const int b = blockIdx.x, h = blockIdx.y;
+  const int b = blockIdx.x;
+  int h = 0;  // the blockIdx.y-th block-sparse head
+  {
+    const HeadStatic* all = at<const HeadStatic>(dp, dp.lay.heads);
+    int seen = -1;
+    for (h = 0; h < dp.Hq; ++h)
+      if (all[h].kind == MSA_BLOCK && ++seen == (int)blockIdx.y) break;
+    if (h >= dp.Hq) return;
+  }
   const HeadStatic& hs = at<const HeadStatic>(dp, dp.lay.heads)[h];
-  if (hs.kind != MSA_BLOCK) return;
   const float* qbar = at<const float>(dp, hs.qbar_off) + (int64_t)b * D;
   const float* kbar = at<const float>(dp, dp.lay.kbar) + (int64_t)hs.kvh * dp.nb * D;
   if (threadIdx.x < D) qb[threadIdx.x] = qbar[threadIdx.x];
@@ -614,11 +664,12 @@ cudaError_t launch_topk_jobs(const DevPlan& dp, cudaStream_t st) {
 
 cudaError_t launch_block_estimate(const DevPlan& dp, const void* Q, const void* K, const msa_strides& s,
                                   cudaStream_t st) {
-  const int gx = std::min(dp.nb, 1024);
-  count_launches(3);
-  pool_kernel<<<dim3(gx, dp.Hkv), D, 0, st>>>(dp, static_cast<const __nv_bfloat16*>(K), s.k_head, s.k_row, dp.Hkv,
-                                              0);
-  pool_kernel<<<dim3(gx, dp.Hq), D, 0, st>>>(dp, static_cast<const __nv_bfloat16*>(Q), s.q_head, s.q_row, dp.Hq, 1);
+  // about eight 256-thread blocks per SM in all, each walking several 64-row blocks
+  const int gx = std::max(1, std::min(dp.nb, sm_count() * 8 / std::max(1, dp.Hkv + dp.n_block_heads)));
+  count_launches(2);
+  pool_kernel<<<dim3(gx, dp.Hkv + dp.n_block_heads), POOL_THREADS, 0, st>>>(
+      dp, static_cast<const __nv_bfloat16*>(Q), s.q_head, s.q_row, static_cast<const __nv_bfloat16*>(K), s.k_head,
+      s.k_row);
   const size_t smem = sizeof(uint32_t) * (size_t)dp.nb;
   static size_t configured = 0;
   if (smem > 48 * 1024 && smem > configured) {
@@ -626,7 +677,7 @@ cudaError_t launch_block_estimate(const DevPlan& dp, const void* Q, const void* 
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  block_topk_kernel<<<dim3(dp.nb, dp.Hq), BT_THREADS, smem, st>>>(dp);
+  block_topk_kernel<<<dim3(dp.nb, std::max(1, dp.n_block_heads)), BT_THREADS, smem, st>>>(dp);
   return cudaGetLastError();
 }
 

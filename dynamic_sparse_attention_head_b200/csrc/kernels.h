@@ -17,6 +17,7 @@ struct DevPlan {
   int32_t x_rows;      // rows per gathered K/V slice
   int32_t n_qslices, n_xslices;
   int32_t has2d, has_block;
+  int32_t n_block_heads;  // query heads of kind MSA_BLOCK
   int32_t nb;          // L / 64
   int64_t n_text;      // text tokens (they lead the modality-grouped order)
   int32_t tb_words;    // unit-bitmap words per tile-builder warp

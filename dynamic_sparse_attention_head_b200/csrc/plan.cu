@@ -578,6 +578,8 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   dp.n_xslices = n_xslices;
   dp.has2d = has2d;
   dp.has_block = has_block;
+  dp.n_block_heads = 0;
+  for (int32_t h = 0; h < Hq; ++h) dp.n_block_heads += prob->heads[h].kind == MSA_BLOCK ? 1 : 0;
   dp.nb = (int32_t)nb;
   dp.n_text = P->n_mod[0];
   dp.scale = P->scale;
