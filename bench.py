@@ -179,7 +179,7 @@ def make_host_inputs(p, seed):
 
 def attn_source_hash():
     h = hashlib.sha256()
-    for f in ("attn.cu", "ptx.cuh", "msa_internal.h"):
+    for f in ("attn.cu", "ptx.cuh", "msa_internal.h", "plan.cu"):  # plan.cu: work-item order
         with open(os.path.join(ROOT, "dynamic_sparse_attention_head_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
