@@ -72,6 +72,7 @@ def _load():
         "msa_read_indices": ([_P, _P, _I32, _P, ctypes.POINTER(_I64), _P], _I32),
         "msa_read_tiles": ([_P, _P, _I32, _P, ctypes.POINTER(_I64), _P], _I32),
         "msa_tile_stats": ([_P, _P, _P, _P], _I32),
+        "msa_attention_units": ([_P, _P], _I32),
         "msa_device_status": ([_P, _P, _P], _I32),
         "msa_status_string": ([_I32], ctypes.c_char_p),
         "msa_kernel_launches": ([], ctypes.c_uint64),
@@ -87,8 +88,8 @@ def _load():
 _lib = _load()
 EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_estimate", "msa_set_indices",
            "msa_permute", "msa_sparse_prefill", "msa_unpermute", "msa_read_indices", "msa_read_tiles",
-           "msa_tile_stats", "msa_device_status", "msa_status_string", "msa_kernel_launches",
-           "msa_vslash_estimate_static")
+           "msa_tile_stats", "msa_attention_units", "msa_device_status", "msa_status_string",
+           "msa_kernel_launches", "msa_vslash_estimate_static")
 
 
 def kernel_launches() -> int:
@@ -311,6 +312,12 @@ class Plan:
     def tile_stats(self, ws, stream=None):
         t = (_I64 * 2)()
         _check("msa_tile_stats", _lib.msa_tile_stats(self._h, ws.data_ptr(), ctypes.cast(t, _P), _stream_ptr(stream)))
+        return int(t[0]), int(t[1])
+
+    def attention_units(self):
+        """(work units, key chunks) of msa_sparse_prefill for this plan."""
+        t = (_I64 * 2)()
+        _check("msa_attention_units", _lib.msa_attention_units(self._h, ctypes.cast(t, _P)))
         return int(t[0]), int(t[1])
 
     def device_status(self, ws, stream=None) -> int:

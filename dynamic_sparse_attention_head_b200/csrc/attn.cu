@@ -40,7 +40,10 @@ struct AttnParams {
   int32_t n_items;
   float scale_log2;        // softmax scale * log2(e)
   float* lse;              // [Hq][L] or null
-  uint32_t* next_item;     // work-item counter, zero at launch
+  uint32_t* next_item;     // work-unit counter, zero at launch
+  int32_t n_units, n_kchunks, n_bands;
+  uint32_t* chunk_done;    // per item: chunks whose state is in its accumulator (chunked keys)
+  float* acc;              // accumulator slots [slot][128][ACC_ROW] (chunked keys)
 };
 
 // warpgroup 0: warps 0 / 2 TMA of stream 0 / 1, warps 1 / 3 MMA of stream 0 / 1; warpgroups
@@ -78,8 +81,10 @@ struct __align__(1024) AttnSmem {
   uint64_t o_full[N_STREAMS], o_free[N_STREAMS];
   // work-item queue of each stream: ids taken from the global counter by the stream's TMA
   // thread, read by its MMA issuer and softmax warpgroup (-1 ends the stream)
-  int32_t iq[N_STREAMS][IQ_DEPTH];
+  int32_t iq[N_STREAMS][IQ_DEPTH][4];  // item, key chunk, accumulator slot
   uint64_t iq_full[N_STREAMS][IQ_DEPTH], iq_empty[N_STREAMS][IQ_DEPTH];
+  // softmax warpgroup handshakes around the accumulator of chunked items
+  uint64_t acc_in[N_STREAMS], acc_out[N_STREAMS];
   uint64_t drain[N_STREAMS];
   RowCtx rctx[256];  // mask state of the row of each softmax thread (read off the critical path)
   uint32_t tmem_base;
@@ -126,6 +131,65 @@ __device__ __forceinline__ bool load_item(const AttnParams& p, int item, ItemInf
   it.x_slice = (int)hs.x_slice;
   if (it.row0 >= it.nrows) it.ntiles = -1;  // no rows: item skipped by every role
   return it.ntiles >= 0;
+}
+
+// One queue entry: the unit's item and key chunk.  it.tile0 / it.ntiles are narrowed to the
+// unit's tiles; k = key chunks of the item before this one that have tiles (their state is in
+// the item's accumulator), last = no tiles of the item after this unit, total = the item's
+// tiles.  False: the item has no rows (every role skips it).
+struct UnitInfo {
+  int item, chunk, acc, k, total;
+  bool last;
+};
+
+__device__ __forceinline__ bool load_unit(const AttnParams& p, const int32_t* e, ItemInfo& it, UnitInfo& u) {
+  u.item = e[0];
+  u.chunk = e[1];
+  u.acc = e[2];
+  if (!load_item(p, u.item, it)) return false;
+  u.total = it.ntiles;
+  u.k = 0;
+  u.last = true;
+  if (p.n_kchunks > 1 && it.ntiles > 0) {
+    const int32_t* cs = reinterpret_cast<const int32_t*>(p.ws + p.lay.cstart) + (int64_t)u.item * (p.n_kchunks + 1);
+    const int t0 = cs[u.chunk], t1 = cs[u.chunk + 1];
+    for (int c = 0; c < u.chunk; ++c) u.k += cs[c + 1] > cs[c] ? 1 : 0;
+    u.last = t1 == it.ntiles;
+    it.tile0 += t0;
+    it.ntiles = t1 - t0;
+  }
+  return true;
+}
+
+// Unit id -> (item, key chunk, accumulator slot).
+__device__ __forceinline__ void unit_entry(const AttnParams& p, int u, int32_t (&e)[3]) {
+  if (p.n_kchunks == 1) {
+    e[0] = u;
+    e[1] = 0;
+    e[2] = -1;
+    return;
+  }
+  const UnitBand* b = reinterpret_cast<const UnitBand*>(p.ws + p.lay.bands);
+  int lo = 0, hi = p.n_bands - 1;  // last band with unit0 <= u
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (b[mid].unit0 <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  const UnitBand bd = b[lo];
+  const int local = u - bd.unit0;
+  e[0] = bd.item0 + local % bd.n;
+  e[1] = local / bd.n;
+  e[2] = bd.acc0 + local % bd.n;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(uint32_t* a, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
 }
 
 
@@ -328,12 +392,14 @@ __device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, ui
   for (uint32_t qi = 0;; ++qi) {
     const uint32_t slot = qi % IQ_DEPTH;
     if (!mbar_wait(&sm.iq_full[s][slot], (qi / IQ_DEPTH) & 1, abort)) return;
-    const int item = sm.iq[s][slot];
+    const int32_t e[3] = {sm.iq[s][slot][0], sm.iq[s][slot][1], sm.iq[s][slot][2]};
     mbar_arrive(&sm.iq_empty[s][slot]);
-    if (item < 0) break;
+    if (e[0] < 0) break;
     ItemInfo it;
-    if (!load_item(p, item, it) || it.ntiles == 0) continue;
+    UnitInfo un;
+    if (!load_unit(p, e, it, un) || it.ntiles == 0) continue;
     const int n = it.ntiles;
+    const bool cont = un.k > 0;  // O starts from the item's accumulator (loaded by the softmax)
     if (!mbar_wait(&sm.q_full[s], q_use & 1, abort)) return;
     ++q_use;
     if (!mbar_wait(&sm.k_full[s], k_use & 1, abort)) return;
@@ -353,7 +419,7 @@ __device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, ui
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // 16 keys per step: 8 TMEM columns of P, 2 KB of V
           umma_ts(s_col + TM_OOFF, s_col + 8 * kk, smem_desc_sw128(v_addr + kk * 2048, ATOM_BYTES, 1024), IDESC_PV,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+                  (cont || j > 0 || kk > 0) ? 1u : 0u);
       }
       umma_commit(&sm.v_empty[s]);
       ++v_use;
@@ -401,6 +467,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         mbar_init(&sm.iq_full[s][i], 1);
         mbar_init(&sm.iq_empty[s][i], IQ_READERS);
       }
+      mbar_init(&sm.acc_in[s], 1);
+      mbar_init(&sm.acc_out[s], 128);
     }
     fence_barrier_init();
   }
@@ -431,10 +499,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       auto publish = [&]() -> bool {
         const uint32_t slot = published % IQ_DEPTH, use = published / IQ_DEPTH;
         if (ended || (use > 0 && !mbar_test(&sm.iq_empty[s][slot], (use - 1) & 1))) return false;
-        int id = (int)atomicAdd(p.next_item, 1u);
-        if (id >= p.n_items) id = -1;
-        ended = id < 0;
-        sm.iq[s][slot] = id;
+        const int id = (int)atomicAdd(p.next_item, 1u);
+        int32_t e[3] = {-1, 0, -1};
+        if (id < p.n_units) unit_entry(p, id, e);
+        ended = e[0] < 0;
+        sm.iq[s][slot][0] = e[0];
+        sm.iq[s][slot][1] = e[1];
+        sm.iq[s][slot][2] = e[2];
         mbar_arrive(&sm.iq_full[s][slot]);
         ++published;
         return true;
@@ -449,9 +520,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (qk_live && qk_op < 0) {  // next item of the Q/K loads
           if (published <= qk_q && publish()) wd.progress();
           if (published > qk_q) {
-            const int id = sm.iq[s][qk_q % IQ_DEPTH];
-            if (id < 0) qk_live = false;
-            else if (!load_item(p, id, qk_it) || qk_it.ntiles == 0) ++qk_q;
+            const int32_t* e = sm.iq[s][qk_q % IQ_DEPTH];
+            UnitInfo un;
+            if (e[0] < 0) qk_live = false;
+            else if (!load_unit(p, e, qk_it, un) || qk_it.ntiles == 0) ++qk_q;
             else qk_op = 0;
           }
         }
@@ -486,11 +558,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         if (v_live && v_j < 0 && published > v_q) {  // next item of the V loads
           const uint32_t slot = v_q % IQ_DEPTH;
-          const int id = sm.iq[s][slot];
-          if (id < 0) {
+          const int32_t* e = sm.iq[s][slot];
+          UnitInfo un;
+          if (e[0] < 0) {
             mbar_arrive(&sm.iq_empty[s][slot]);
             v_live = false;
-          } else if (!load_item(p, id, v_it) || v_it.ntiles == 0) {
+          } else if (!load_unit(p, e, v_it, un) || v_it.ntiles == 0) {
             mbar_arrive(&sm.iq_empty[s][slot]);
             ++v_q;
           } else {
@@ -536,16 +609,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t s_own = lane_base, o_own = lane_base + TM_OOFF;
     __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(p.ws + p.lay.op));
     const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
-    uint32_t s_count = 0, items_done = 0;
+    uint32_t s_count = 0, items_done = 0, acc_ins = 0, acc_outs = 0;
     bool ok = true;
     for (uint32_t qi = 0; ok; ++qi) {
       const uint32_t slot = qi % IQ_DEPTH;
       if (!mbar_wait(&sm.iq_full[s][slot], (qi / IQ_DEPTH) & 1, abort)) break;
-      const int item = sm.iq[s][slot];
+      const int32_t e[3] = {sm.iq[s][slot][0], sm.iq[s][slot][1], sm.iq[s][slot][2]};
       mbar_arrive(&sm.iq_empty[s][slot]);
-      if (item < 0) break;
+      if (e[0] < 0) break;
       ItemInfo it;
-      if (!load_item(p, item, it)) continue;
+      UnitInfo un;
+      if (!load_unit(p, e, it, un)) continue;
+      if (un.total > 0 && it.ntiles == 0) continue;  // no keys of this item in this chunk
+      if (un.total == 0 && un.chunk != 0) continue;  // an item without tiles is written once
       const ClassStatic& cs = class_of(p, it.cls);
       const int r = it.row0 + t;
       RowCtx& rc = sm.rctx[threadIdx.x - 128];
@@ -579,6 +655,40 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
 
       float m_used = -INFINITY, l = 0.f;
+      // A unit after the item's first key chunk resumes from the item's accumulator: the
+      // previous chunk's unit releases it (chunk_done) once every row is stored.
+      const bool cont = un.k > 0;
+      float* arow = p.acc ? p.acc + ((int64_t)un.acc * TILE + t) * ACC_ROW : nullptr;
+      if (cont) {
+        if (t == 0) {
+          const uint64_t t0 = global_ns();
+          while (ld_acquire(p.chunk_done + un.item) < (uint32_t)un.k) {
+            if (*abort || global_ns() - t0 > 1000000000ull) {
+              *abort = 1;
+              break;
+            }
+          }
+          mbar_arrive(&sm.acc_in[s]);
+        }
+        if (!mbar_wait(&sm.acc_in[s], acc_ins & 1, abort)) { ok = false; break; }
+        ++acc_ins;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t oa[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(arow + 32 * c + 4 * j));
+            oa[4 * j] = __float_as_uint(v.x);
+            oa[4 * j + 1] = __float_as_uint(v.y);
+            oa[4 * j + 2] = __float_as_uint(v.z);
+            oa[4 * j + 3] = __float_as_uint(v.w);
+          }
+          tmem_st32(o_own + 32 * c, oa);
+        }
+        m_used = __ldcg(arow + D);
+        l = __ldcg(arow + D + 1);
+        tmem_wait_st();
+      }
       // The element mask of a tile is built before its S is waited for (for the first tile
       // here, for the others right after the previous tile's P is handed over), so that the
       // bitmap loads and the bit arithmetic overlap the tensor core's work.  Tiles flagged full
@@ -634,7 +744,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         // S_s(tt) complete implies the previous P V of this stream is complete (same issuer,
         // issue order), so O_s may be rescaled here
-        if (tt > 0 && __any_sync(0xFFFFFFFFu, resc)) {
+        if ((tt > 0 || cont) && __any_sync(0xFFFFFFFFu, resc)) {
           const float f = resc ? alpha : 1.f;
 #pragma unroll 1
           for (int c = 0; c < 8; ++c) {  // 16 columns at a time: S stays live in registers
@@ -670,10 +780,38 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (tt + 1 < it.ntiles) build_mask(tile_next);
       }
       if (!ok) break;
-      // epilogue: the item's last P V done, then O = O_s / l
+      // epilogue: the unit's last P V done, then O = O_s / l, or the state into the accumulator
       if (!mbar_wait(&sm.o_full[s], items_done & 1, abort)) { ok = false; break; }
       ++items_done;
       tc_fence_after();
+      if (!un.last) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t oa[32];
+          tmem_ld32(o_own + 32 * c, oa);
+          tmem_wait_ld();
+          if (c == 3) {
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[s]);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            __stcg(reinterpret_cast<float4*>(arow + 32 * c + 4 * j),
+                   make_float4(__uint_as_float(oa[4 * j]), __uint_as_float(oa[4 * j + 1]),
+                               __uint_as_float(oa[4 * j + 2]), __uint_as_float(oa[4 * j + 3])));
+        }
+        __stcg(arow + D, m_used);
+        __stcg(arow + D + 1, l);
+        __threadfence();
+        mbar_arrive(&sm.acc_out[s]);
+        if (t == 0) {
+          if (!mbar_wait(&sm.acc_out[s], acc_outs & 1, abort)) { ok = false; break; }
+          __threadfence();
+          st_release(p.chunk_done + un.item, (uint32_t)un.k + 1u);
+        }
+        ++acc_outs;
+        continue;
+      }
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint4* dst = reinterpret_cast<uint4*>(op + orow);
 #pragma unroll
@@ -773,6 +911,16 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
   // work items are handed out by a counter in the workspace header, zeroed here
   p.next_item = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(ws + dp.lay.header)) + HDR_NEXT_ITEM;
   if (cudaError_t e = cudaMemsetAsync(p.next_item, 0, sizeof(uint32_t), st)) return e;
+  p.n_units = dp.n_units;
+  p.n_kchunks = dp.n_kchunks;
+  p.n_bands = dp.n_bands;
+  p.chunk_done = nullptr;
+  p.acc = nullptr;
+  if (dp.n_kchunks > 1) {
+    p.chunk_done = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(ws + dp.lay.chunk_done));
+    p.acc = reinterpret_cast<float*>(const_cast<uint8_t*>(ws + dp.lay.acc));
+    if (cudaError_t e = cudaMemsetAsync(p.chunk_done, 0, sizeof(uint32_t) * (size_t)dp.n_items, st)) return e;
+  }
   const size_t smem = sizeof(AttnSmem);
   static bool configured = false;
   if (!configured) {
@@ -780,7 +928,7 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int grid = std::max(1, std::min((dp.n_items + N_STREAMS - 1) / N_STREAMS, sm_count()));
+  const int grid = std::max(1, std::min((dp.n_units + N_STREAMS - 1) / N_STREAMS, sm_count()));
   count_launches(1);
   msa_attn_kernel<<<grid, ATT_THREADS, smem, st>>>(mq, mqp, mk, mv, mk2, mv2, mxk, mxv, p);
   return cudaGetLastError();

@@ -470,6 +470,8 @@ __global__ void __launch_bounds__(TB_WARPS * 32) tiles_kernel(DevPlan dp, int bm
     const int row0 = wi.slot * TILE;
     if (row0 >= nrows) {
       if (lane == 0) ntiles[item] = 0;
+      if (dp.n_kchunks > 1)
+        for (int c = lane; c <= dp.n_kchunks; c += 32) at<int32_t>(dp, dp.lay.cstart)[(int64_t)item * (dp.n_kchunks + 1) + c] = 0;
       continue;
     }
     const int nval = min(TILE, nrows - row0);
@@ -504,6 +506,8 @@ __global__ void __launch_bounds__(TB_WARPS * 32) tiles_kernel(DevPlan dp, int bm
         flag_bounds(dp);
         ntiles[item] = 0;
       }
+      if (dp.n_kchunks > 1)
+        for (int c = lane; c <= dp.n_kchunks; c += 32) at<int32_t>(dp, dp.lay.cstart)[(int64_t)item * (dp.n_kchunks + 1) + c] = 0;
       continue;
     }
     for (int w = lane; w < wmax; w += 32) bm[w] = 0u;
@@ -623,6 +627,23 @@ __global__ void __launch_bounds__(TB_WARPS * 32) tiles_kernel(DevPlan dp, int bm
         }
       }
       if (full) out[i] = t | TILE_FULL;
+    }
+    __syncwarp();
+    // ---- first tile of each key chunk (gathered-key tiles count as chunk 0; the list is in
+    // chunk order: gathered tiles first, then identity windows by ascending key row)
+    if (dp.n_kchunks > 1) {
+      int32_t* cst = at<int32_t>(dp, dp.lay.cstart) + (int64_t)item * (dp.n_kchunks + 1);
+      for (int c = lane; c <= dp.n_kchunks; c += 32) {
+        int lo = 0, hi = nt;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          const uint32_t t = out[mid];
+          const int tc = ((t >> 28) == SRC_X) ? 0 : (int)((t & TILE_ROW_MASK) / dp.chunk_keys);
+          if (tc < c) lo = mid + 1;
+          else hi = mid;
+        }
+        cst[c] = (c == dp.n_kchunks) ? nt : lo;
+      }
     }
     __syncwarp();
   }

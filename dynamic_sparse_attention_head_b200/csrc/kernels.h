@@ -14,6 +14,10 @@ struct DevPlan {
   int64_t L;
   int32_t Hq, Hkv, LP;
   int32_t n_classes, n_heads, n_rowsets, n_jobs, n_items, n_segs;
+  int32_t n_units;     // attention work units (= n_items when the keys are not chunked)
+  int32_t n_kchunks;   // key chunks of the attention kernel (1: not chunked)
+  int32_t chunk_keys;  // keys per chunk (a multiple of 128)
+  int32_t n_bands;     // unit bands (chunked keys only)
   int32_t x_rows;      // rows per gathered K/V slice
   int32_t n_qslices, n_xslices;
   int32_t has2d, has_block;

@@ -129,6 +129,21 @@ struct WorkItem {
   int32_t cls, slot;         // class, 128-row slot within the class
 };
 
+// Units of work of the attention kernel when the keys are chunked: the tiles of one work item
+// whose keys lie in one key chunk (gathered-key tiles count as chunk 0).  The work items are cut
+// into bands (consecutive items of the plan order); a band's units run chunk-major, so that the
+// units in flight read one chunk of K/V, and a long item carries its online-softmax state
+// (unnormalised O, running max and sum) from chunk to chunk through an accumulator slot.
+// Band b holds items [item0, item0 + n) and units [unit0, unit0 + n * n_kchunks): unit
+// unit0 + c n + i is chunk c of item item0 + i, accumulator slot acc0 + i.
+struct UnitBand {
+  int32_t item0, n, acc0, unit0;
+};
+// fp32 per accumulator row: O[128], running max (log2), running sum, padding to a multiple of
+// four so that every row starts on a 16-byte boundary (rows are moved with 16-byte accesses)
+constexpr int ACC_ROW = D + 4;
+static_assert(ACC_ROW % 4 == 0, "accumulator rows must be 16-byte aligned");
+
 // Byte offsets of the workspace regions.
 struct Layout {
   int64_t header;            // uint32 [64]: [0] error bits, [1] ready flags, [2] attention work-item counter, [8..] stats
@@ -140,6 +155,10 @@ struct Layout {
   int64_t segs;              // int32 [n_segments][3] start, len, modality
   int64_t class_dyn;         // ClassDyn [n_classes]
   int64_t item_ntiles;       // int32 [n_items]
+  int64_t bands;             // UnitBand [n_bands] (chunked keys only)
+  int64_t cstart;            // int32 [n_items][n_kchunks + 1]: first tile of each key chunk (chunked keys only)
+  int64_t chunk_done;        // uint32 [n_items]: chunks of the item whose state is in its accumulator
+  int64_t acc;               // fp32 [n_acc][128][ACC_ROW]: per-item online-softmax state between chunks
   int64_t tiles;             // uint32 [total tile capacity]: (src << 28) | TILE_FULL? | first key row
   int64_t modality;          // uint8 [L]
   int64_t rank;              // int32 [L]

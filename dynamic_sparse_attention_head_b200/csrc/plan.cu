@@ -6,7 +6,9 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
+#include <tuple>
 #include <new>
 #include <vector>
 
@@ -36,9 +38,11 @@ struct msa_plan {
   std::vector<RowSet> rowsets;
   std::vector<TopkJob> jobs;
   std::vector<WorkItem> items;
+  std::vector<UnitBand> bands;
   std::vector<int32_t> segtab;
   Layout lay{};
   DevPlan dp{};
+  int32_t n_kchunks = 1, chunk_keys = 0, n_units = 0, band_cap = 0;
   int64_t blob_bytes = 0;
   std::vector<uint8_t> blob;
   int64_t total_tiles = 0;
@@ -319,6 +323,47 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
             for (int c = 0; c < (int)C.size(); ++c)
               if (C[c].kvh == g && C[c].k_src == src && prob->heads[C[c].head].kind == kind && s < C[c].n_items)
                 P->items.push_back(WorkItem{c, s});
+    // ---- key chunks of the attention kernel: when one head's K and V (L x 512 B) no longer fit
+    // comfortably in L2, the keys are cut into 64K-key chunks (32 MB of K and V per head); the
+    // environment variable MSA_ATTN_CHUNK_KEYS (a multiple of 128) overrides the chunk size.
+    int64_t ck = (int64_t)L * 512 > (96ll << 20) ? 65536 : 0;
+    if (const char* env = std::getenv("MSA_ATTN_CHUNK_KEYS")) ck = std::max<int64_t>(0, std::atoll(env)) / TILE * TILE;
+    P->n_kchunks = (ck > 0 && ck < L) ? (int32_t)((L + ck - 1) / ck) : 1;
+    P->chunk_keys = P->n_kchunks > 1 ? (int32_t)ck : (int32_t)L;
+    P->bands.clear();
+    P->band_cap = 0;
+    if (P->n_kchunks > 1) {
+      // bands: runs of the plan order within one (KV head, key source, head kind) group and one
+      // range of 1024 slots, merged until each holds at least 2048 units, so that no more than
+      // two bands have units in flight (a stream holds at most five) and two accumulator
+      // buffers, used by alternate bands, suffice
+      constexpr int32_t BAND_SLOTS = 1024, MIN_UNITS = 2048;
+      auto key = [&](const WorkItem& w) {
+        const ClassStatic& c = C[w.cls];
+        return std::make_tuple(c.kvh, c.k_src, prob->heads[c.head].kind, w.slot / BAND_SLOTS);
+      };
+      int32_t i0 = 0;
+      const int32_t n = (int32_t)P->items.size();
+      int64_t unit0 = 0;
+      for (int32_t i = 1; i <= n; ++i) {
+        const bool cut = i == n || key(P->items[i]) != key(P->items[i - 1]);
+        if (!cut) continue;
+        if (i < n && (int64_t)(i - i0) * P->n_kchunks < MIN_UNITS) continue;  // merge into the next run
+        UnitBand b{i0, i - i0, 0, (int32_t)unit0};
+        P->bands.push_back(b);
+        unit0 += (int64_t)b.n * P->n_kchunks;
+        P->band_cap = std::max(P->band_cap, b.n);
+        i0 = i;
+      }
+      for (size_t b = 0; b < P->bands.size(); ++b) P->bands[b].acc0 = (int32_t)(b & 1) * P->band_cap;
+      if (unit0 > INT32_MAX) {
+        delete P;
+        return MSA_ERR_UNSUPPORTED;
+      }
+      P->n_units = (int32_t)unit0;
+    } else {
+      P->n_units = (int32_t)P->items.size();
+    }
     int64_t tb = 0;
     for (auto& c : C) {
       c.tile_base = tb;
@@ -415,10 +460,16 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   const int64_t max_jobs = (int64_t)RS.size() * 3 + 1;
   lay.jobs = B.take((int64_t)sizeof(TopkJob) * max_jobs);
   lay.items = B.take((int64_t)sizeof(WorkItem) * P->items.size());
+  lay.bands = B.take((int64_t)sizeof(UnitBand) * std::max<size_t>(P->bands.size(), 1));
   lay.segs = B.take(4 * (int64_t)P->segtab.size());
   P->blob_bytes = B.off;
   lay.class_dyn = B.take((int64_t)sizeof(ClassDyn) * C.size());
   lay.item_ntiles = B.take(4 * (int64_t)P->items.size());
+  if (P->n_kchunks > 1) {
+    lay.cstart = B.take(4 * (int64_t)P->items.size() * (P->n_kchunks + 1));
+    lay.chunk_done = B.take(4 * (int64_t)P->items.size());
+    lay.acc = B.take(4 * 2 * (int64_t)P->band_cap * TILE * ACC_ROW, 1024);
+  }
   lay.tiles = B.take(4 * P->total_tiles);
   lay.modality = B.take(L);
   lay.rank = B.take(4 * L);
@@ -558,6 +609,7 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   if (!RS.empty()) std::memcpy(P->blob.data() + lay.rowsets, RS.data(), sizeof(RowSet) * RS.size());
   if (!P->jobs.empty()) std::memcpy(P->blob.data() + lay.jobs, P->jobs.data(), sizeof(TopkJob) * P->jobs.size());
   std::memcpy(P->blob.data() + lay.items, P->items.data(), sizeof(WorkItem) * P->items.size());
+  if (!P->bands.empty()) std::memcpy(P->blob.data() + lay.bands, P->bands.data(), sizeof(UnitBand) * P->bands.size());
   std::memcpy(P->blob.data() + lay.segs, P->segtab.data(), 4 * P->segtab.size());
 
   DevPlan& dp = P->dp;
@@ -572,6 +624,10 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   dp.n_rowsets = (int32_t)RS.size();
   dp.n_jobs = (int32_t)P->jobs.size();
   dp.n_items = (int32_t)P->items.size();
+  dp.n_units = P->n_units;
+  dp.n_kchunks = P->n_kchunks;
+  dp.chunk_keys = P->chunk_keys;
+  dp.n_bands = (int32_t)P->bands.size();
   dp.n_segs = (int32_t)P->segs.size();
   dp.x_rows = std::max(x_rows_max, TILE);
   dp.n_qslices = n_qslices;
@@ -797,6 +853,13 @@ msa_status msa_device_status(const msa_plan* P, void* ws, void* stream) {
   }
   if (err & DEV_ERR_TIMEOUT) return MSA_ERR_TIMEOUT;
   if (err & DEV_ERR_BOUNDS) return MSA_ERR_DEVICE_BOUNDS;
+  return MSA_OK;
+}
+
+msa_status msa_attention_units(const msa_plan* P, int64_t out[2]) {
+  if (!P || !out) return MSA_ERR_INVALID_ARG;
+  out[0] = P->n_units;
+  out[1] = P->n_kchunks;
   return MSA_OK;
 }
 

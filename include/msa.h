@@ -191,6 +191,15 @@ msa_status msa_read_indices(const msa_plan* plan, const void* ws, int32_t head, 
  * Executed block FLOPs = 4 * 128 * 128 * 128 * tiles[0]. */
 msa_status msa_tile_stats(const msa_plan* plan, const void* ws, int64_t tiles[2], void* stream);
 
+/* How msa_sparse_prefill divides its work (host only, no device access): out[0] = work units,
+ * out[1] = key chunks.  When one head's K and V exceed about 96 MB (L > 192K tokens) the keys
+ * are cut into chunks of 65536 (the environment variable MSA_ATTN_CHUNK_KEYS, a multiple of
+ * 128, read at msa_plan_create, overrides the chunk size; 0 turns chunking off): the units of a
+ * band of work items then run chunk by chunk so that the units in flight share one chunk of
+ * K and V in L2, and a work item's online-softmax state passes from chunk to chunk through an
+ * accumulator in the workspace.  The result does not depend on the chunking beyond rounding. */
+msa_status msa_attention_units(const msa_plan* plan, int64_t out[2]);
+
 /* Dumps the work list of head `head` for tests: for each of its 128-query work items the
  * query positions covered (-1 for padding) and, for every executed tile, its key source
  * (0 = keys in original order, 1 = modality-grouped keys, 2 = gathered keys; plus 8 when every

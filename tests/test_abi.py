@@ -61,3 +61,20 @@ def test_workspace_grows_with_length():
     a = msa.Plan(llama3_8b_text(L=4096)).workspace_bytes
     b = msa.Plan(llama3_8b_text(L=8192)).workspace_bytes
     assert b > a
+
+
+def test_attention_units_chunking_rule(monkeypatch):
+    """Keys are chunked (65536 per chunk) only when one head's K and V exceed ~96 MB; the
+    environment override applies at plan creation."""
+    import dynamic_sparse_attention_head_b200 as msa
+    import workload
+    monkeypatch.delenv("MSA_ATTN_CHUNK_KEYS", raising=False)
+    assert msa.Plan(workload.qwen2_7b_video_128k()).attention_units()[1] == 1
+    units, chunks = msa.Plan(workload.longvila_1m()).attention_units()
+    assert chunks == 16
+    monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", "256")
+    p = workload.llama3_8b_text(L=2048)
+    assert msa.Plan(p).attention_units()[1] == 8
+    monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", "0")
+    units, chunks = msa.Plan(p).attention_units()
+    assert chunks == 1
