@@ -40,6 +40,7 @@ def workloads():
         "llama3-8b-text-32k": lambda: workload.llama3_8b_text(L=32768),
         "grid-1head-4k": lambda: workload.grid_single_head(),
         "qwen2-7b-video-64f": workload.qwen2_7b_video_literal,
+        "mixed-image-text-64k": lambda: workload.mixed_image_text(L=65536),
     }
     for L in workload.SWEEP_LENGTHS:
         W[f"sweep-dense-L{L}"] = (lambda L=L: workload.sweep_layer(L, None))

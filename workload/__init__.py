@@ -220,6 +220,35 @@ def qwen2_7b_video_literal() -> Problem:
     return qwen2_7b_video(frames_per_run=[22, 21, 21], texts=(2048, 2048, 2048), name="qwen2-7b-video-64f")
 
 
+def mixed_image_text(L: int = 65536, image: int = 576, width: int = 24, text: Tuple[int, int] = (32, 640),
+                     k_v: int = 1000, k_s: int = 6096, grid_budget: float = 0.10, Hq: int = 28, Hkv: int = 4,
+                     seed: int = 0, name: str = "") -> Problem:
+    """A multi-image document: images of `image` patch tokens (rows of `width` tokens) alternate
+    with text runs of seeded random length in [text[0], text[1]], the last run filling up to L;
+    many short segments of both modalities stress the Q- and 2D-boundary heads (row-class and
+    modality-grouped tiles cut at every segment edge).  Head kinds Q-boundary, 2D-boundary,
+    vertical-slash and grid (stride = image row width)."""
+    rng = np.random.default_rng(seed)
+    segs, pos = [], 0
+    while True:
+        if pos + image + text[0] > L:
+            break
+        segs.append((pos, image, VIDEO)); pos += image
+        n = int(rng.integers(text[0], text[1] + 1))
+        n = min(n, L - pos) if L - pos - n < image + text[0] else n
+        segs.append((pos, n, TEXT)); pos += n
+    if pos < L:
+        if segs and segs[-1][2] == TEXT:
+            s0, n0, _ = segs.pop()
+            segs.append((s0, n0 + (L - pos), TEXT))
+        else:
+            segs.append((pos, L - pos, TEXT))
+    kinds = [Head("qbound", k_v=k_v, k_s=k_s), Head("bound2d", k_v=k_v, k_s=k_s), Head("vslash", k_v=k_v, k_s=k_s),
+             Head("grid", strides=(width,), grid_budget=grid_budget)]
+    return Problem(L=L, Hq=Hq, Hkv=Hkv, segments=segs, heads=_assign(Hq, kinds), frame_stride=width,
+                   name=name or f"mixed-image-text-L{L}")
+
+
 def longvila_1m(L: int = 1048576, stride: int = 256, text: int = 512, grid_budget: float = 0.05,
                 k_v: int = 1000, k_s: int = 6096, Hq: int = 28, Hkv: int = 4) -> Problem:
     """LongVILA-1M-like layer: video frames of `stride` tokens then one trailing text query."""
