@@ -277,36 +277,63 @@ def run_ours(args, rank, world, local_rank):
     ms_step = total_ms / args.steps
     value = job_flops * args.steps / (total_ms * 1e-3) / 1e12
 
-    # end to end through the public API with host buffers: H2D inputs, path, D2H output
+    # end to end through the public API with host buffers: every step copies its Q/K/V from
+    # pinned host memory, runs the path and reads its O back to pinned host memory.  The copies
+    # are pipelined across steps as a caller streaming layers would: two device buffer sets, the
+    # H2D copy of step s+1 and the D2H copy of step s-1 run on copy streams while step s
+    # computes; the timed region spans the first H2D copy to the last D2H copy.
     e2e = None
     if not args.no_e2e:
         qp = torch.from_numpy(Qh).view(torch.bfloat16).pin_memory()
         kp = torch.from_numpy(Kh).view(torch.bfloat16).pin_memory()
         vp = torch.from_numpy(Vh).view(torch.bfloat16).pin_memory()
-        op = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+        ohost = [torch.empty(o.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        bufs = [(q, k, v, o), tuple(torch.empty_like(x) for x in (q, k, v, o))]
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
+        in_ready, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-        def e2e_step():
-            q.copy_(qp, non_blocking=True)
-            k.copy_(kp, non_blocking=True)
-            v.copy_(vp, non_blocking=True)
-            step()
-            op.copy_(o, non_blocking=True)
+        def run_e2e(n):
+            for s_ in range(n):
+                b = s_ % 2
+                bq, bk, bv, bo = bufs[b]
+                with torch.cuda.stream(h2d):
+                    if s_ >= 2:
+                        h2d.wait_event(comp_done[b])  # step s-2 is done with this buffer set
+                    bq.copy_(qp, non_blocking=True)
+                    bk.copy_(kp, non_blocking=True)
+                    bv.copy_(vp, non_blocking=True)
+                    in_ready[b].record(h2d)
+                stream.wait_event(in_ready[b])
+                if s_ >= 2:
+                    stream.wait_event(out_done[b])  # O of step s-2 has reached the host
+                plan.estimate(bq, bk, ws)
+                plan.permute(bq, bk, bv, ws)
+                plan.sparse_prefill(bq, bk, bv, ws)
+                plan.unpermute(ws, bo)
+                comp_done[b].record(stream)
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(comp_done[b])
+                    ohost[b].copy_(bo, non_blocking=True)
+                    out_done[b].record(d2h)
 
-        e2e_step()
+        run_e2e(2)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        h2d.wait_event(s0)
+        run_e2e(args.steps)
+        stream.wait_stream(d2h)
         s1.record(stream)
         torch.cuda.synchronize()
         e2e_ms, _ = job_totals(s0.elapsed_time(s1), 0.0, world, dev)
         bi = (Qh.nbytes + Kh.nbytes + Vh.nbytes)
         bo = int(np.prod(o.shape)) * 2
         e2e = {"value": job_flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps}
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps,
+               "copies": "pipelined across steps (two device buffer sets, H2D and D2H streams)"}
 
     pk, pk_src = peaks()
     attn_ms = float(stage[:, 2].mean())
