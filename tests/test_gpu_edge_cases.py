@@ -1,0 +1,108 @@
+"""Degenerate and edge inputs through the C ABI against the oracle: the shortest sequences (one
+partial tile), rows the mask leaves empty (O = 0, LSE = -inf), sequence-major [L, H, d] tensors
+passed through explicit strides, no GQA and one KV head for many query heads, and layouts with a
+single modality under the modality-aware heads."""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import compare_outputs, to_dev
+from test_gpu_estimate import _check_head
+from workload import TEXT, VIDEO, Head, Problem, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import dynamic_sparse_attention_head_b200 as msa  # noqa: E402
+
+ALL_KINDS = [Head("dense"), Head("ashape", sink=16, local=40), Head("vslash", k_v=8, k_s=16),
+             Head("block", topk_blocks=2), Head("grid", strides=(32,), grid_budget=0.25),
+             Head("qbound", k_v=8, k_s=16), Head("bound2d", k_v=8, k_s=16)]
+
+
+def _forward(p, Q, K, V, q=None, k=None, v=None, o=None):
+    plan = msa.Plan(p)
+    ws = plan.alloc_workspace()
+    q = to_dev(Q) if q is None else q
+    k = to_dev(K) if k is None else k
+    v = to_dev(V) if v is None else v
+    o = torch.empty((p.Hq, p.L, 128), dtype=torch.bfloat16, device="cuda") if o is None else o
+    lse = torch.empty((p.Hq, p.L), dtype=torch.float32, device="cuda")
+    plan.forward(q, k, v, ws, o, lse=lse)
+    torch.cuda.synchronize()
+    assert plan.device_status(ws) == 0
+    idx = [plan.read_indices(h, ws) for h in range(p.Hq)]
+    return idx, o, lse.cpu().numpy()
+
+
+def _check(p, Q, K, V, idx, o, lse, what):
+    for h in range(p.Hq):
+        _check_head(p, h, idx[h], oracle.estimate_head(p, h, Q, K))
+    Oref, lref = oracle.attention(p, Q, K, V, idx)
+    got = o.float().cpu().numpy()
+    for h in range(p.Hq):
+        compare_outputs(got[h], Oref[h], f"{what} head {h}")
+        fin = np.isfinite(lref[h])
+        assert np.array_equal(fin, np.isfinite(lse[h])), f"{what} head {h}: empty rows differ"
+        np.testing.assert_allclose(lse[h][fin], lref[h][fin], atol=2e-3, rtol=1e-3)
+    return Oref, lref
+
+
+@pytest.mark.parametrize("L", [64, 128, 192])
+def test_shortest_sequences_every_kind(L):
+    segs = [(0, L // 2, VIDEO), (L // 2, L - L // 2, TEXT)] if L >= 128 else [(0, L, VIDEO)]
+    p = Problem(L=L, Hq=len(ALL_KINDS), Hkv=1, segments=segs, heads=ALL_KINDS, frame_stride=32, name=f"L{L}")
+    Q, K, V = make_inputs(p, seed=L)
+    idx, o, lse = _forward(p, Q, K, V)
+    _check(p, Q, K, V, idx, o, lse, f"L={L}")
+
+
+def test_rows_left_empty_give_zero_output():
+    # one vertical and one slash line: most early rows see neither (no entries are forced)
+    p = Problem(L=512, Hq=2, Hkv=1, segments=[(0, 512, TEXT)],
+                heads=[Head("vslash", k_v=1, k_s=1), Head("block", topk_blocks=1)], name="empty-rows")
+    Q, K, V = make_inputs(p, seed=3)
+    idx, o, lse = _forward(p, Q, K, V)
+    Oref, lref = _check(p, Q, K, V, idx, o, lse, "empty rows")
+    empty = ~np.isfinite(lref[0])
+    assert empty.any(), "the layout leaves some rows without keys"
+    assert np.all(o[0].float().cpu().numpy()[empty] == 0.0)
+
+
+def test_sequence_major_tensors_through_strides():
+    p = Problem(L=1088, Hq=4, Hkv=2, segments=[(0, 512, VIDEO), (512, 576, TEXT)],
+                heads=[Head("qbound", k_v=20, k_s=50), Head("grid", strides=(64,), grid_budget=0.2),
+                       Head("vslash", k_v=30, k_s=60), Head("ashape", sink=32, local=100)],
+                frame_stride=64, name="seq-major")
+    Q, K, V = make_inputs(p, seed=6)
+    lhd = lambda x: to_dev(x).permute(1, 0, 2).contiguous()  # noqa: E731  [L, H, d] buffers
+    q, k, v = lhd(Q), lhd(K), lhd(V)
+    o = torch.empty((p.L, p.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    idx, _, lse = _forward(p, Q, K, V, q.permute(1, 0, 2), k.permute(1, 0, 2), v.permute(1, 0, 2),
+                           o.permute(1, 0, 2))
+    _check(p, Q, K, V, idx, o.permute(1, 0, 2), lse, "seq-major")
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 1)])
+def test_group_sizes(hq, hkv):
+    kinds = [Head("vslash", k_v=16, k_s=40), Head("block", block_budget=0.3), Head("ashape", sink=8, local=64),
+             Head("dense")]
+    p = Problem(L=704, Hq=hq, Hkv=hkv, segments=[(0, 704, TEXT)], heads=[kinds[h % 4] for h in range(hq)],
+                name=f"g{hq}x{hkv}")
+    Q, K, V = make_inputs(p, seed=hq + hkv)
+    idx, o, lse = _forward(p, Q, K, V)
+    _check(p, Q, K, V, idx, o, lse, p.name)
+
+
+@pytest.mark.parametrize("modality", [VIDEO, TEXT])
+def test_single_modality_layout(modality):
+    p = Problem(L=1024, Hq=3, Hkv=1, segments=[(0, 1024, modality)],
+                heads=[Head("qbound", k_v=16, k_s=40), Head("bound2d", k_v=16, k_s=40),
+                       Head("grid", strides=(64,), grid_budget=0.2) if modality == VIDEO else Head("vslash", k_v=16, k_s=40)],
+                frame_stride=64 if modality == VIDEO else 0, name=f"only-{modality}")
+    Q, K, V = make_inputs(p, seed=9)
+    idx, o, lse = _forward(p, Q, K, V)
+    _check(p, Q, K, V, idx, o, lse, p.name)
