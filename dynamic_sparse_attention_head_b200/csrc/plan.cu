@@ -316,13 +316,22 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
       c.tile_cap = (int32_t)(c.x_cap / TILE + (nunits + 1) / 2);
     }
     for (int c = 0; c < (int)C.size(); ++c) C[c].item0 = -1;
-    for (int32_t g = 0; g < prob->Hkv; ++g)
-      for (int32_t src : {SRC_K, SRC_K2D})  // K/V in original order, then the modality-grouped copy
-        for (int32_t kind = MSA_DENSE; kind <= MSA_BOUND2D; ++kind)
-          for (int32_t s = max_slots - 1; s >= 0; --s)
-            for (int c = 0; c < (int)C.size(); ++c)
-              if (C[c].kvh == g && C[c].k_src == src && prob->heads[C[c].head].kind == kind && s < C[c].n_items)
-                P->items.push_back(WorkItem{c, s});
+    // when every head's K and V fit in L2 together (about half of it), the grouping buys no
+    // reuse and only delays the last group's longest items: plain longest-first order then
+    const bool group = (int64_t)Hkv * L * 512 * (has2d ? 2 : 1) > (64ll << 20);
+    if (group) {
+      for (int32_t g = 0; g < prob->Hkv; ++g)
+        for (int32_t src : {SRC_K, SRC_K2D})  // K/V in original order, then the modality-grouped copy
+          for (int32_t kind = MSA_DENSE; kind <= MSA_BOUND2D; ++kind)
+            for (int32_t s = max_slots - 1; s >= 0; --s)
+              for (int c = 0; c < (int)C.size(); ++c)
+                if (C[c].kvh == g && C[c].k_src == src && prob->heads[C[c].head].kind == kind && s < C[c].n_items)
+                  P->items.push_back(WorkItem{c, s});
+    } else {
+      for (int32_t s = max_slots - 1; s >= 0; --s)
+        for (int c = 0; c < (int)C.size(); ++c)
+          if (s < C[c].n_items) P->items.push_back(WorkItem{c, s});
+    }
     // ---- key chunks of the attention kernel: when one head's K and V (L x 512 B) no longer fit
     // comfortably in L2, the keys are cut into 64K-key chunks (32 MB of K and V per head); the
     // environment variable MSA_ATTN_CHUNK_KEYS (a multiple of 128) overrides the chunk size.
