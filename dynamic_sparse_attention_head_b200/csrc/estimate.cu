@@ -196,25 +196,36 @@ __global__ void __launch_bounds__(LQ_THREADS) lastq_pass1(DevPlan dp, const __nv
     __syncthreads();
     float c[8][4];
     block_logits(sm, b & 1, af, c);
+    // the block's logits of both rows (log2 units; -inf where not causal), the rows' block
+    // maxima over the quad, then one rescale of the running sums and one exp2 per element
+    float bm0 = -INFINITY, bm1 = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int col = nt * 8 + 2 * t + (e & 1);
-        const int32_t kp = sm.kpos[b & 1][col];
+        const int32_t kp = sm.kpos[b & 1][nt * 8 + 2 * t + (e & 1)];
         const bool top = e < 2;
-        const int32_t rp = top ? p0 : p1;
-        if (kp > rp) continue;
-        const float x = (c[nt][e] * dp.scale) * LOG2E;
-        float& m = top ? m0 : m1;
-        float& z = top ? z0 : z1;
-        if (x > m) {
-          z = z * ex2(m - x) + 1.f;
-          m = x;
-        } else {
-          z += ex2(x - m);
-        }
+        const float x = (kp > (top ? p0 : p1)) ? -INFINITY : (c[nt][e] * dp.scale) * LOG2E;
+        c[nt][e] = x;
+        if (top) bm0 = fmaxf(bm0, x);
+        else bm1 = fmaxf(bm1, x);
       }
+    }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      bm0 = fmaxf(bm0, __shfl_xor_sync(0xFFFFFFFFu, bm0, o));
+      bm1 = fmaxf(bm1, __shfl_xor_sync(0xFFFFFFFFu, bm1, o));
+    }
+    const float n0 = fmaxf(m0, bm0), n1 = fmaxf(m1, bm1);
+    if (n0 > -INFINITY) z0 = (m0 == -INFINITY) ? 0.f : z0 * ex2(m0 - n0);
+    if (n1 > -INFINITY) z1 = (m1 == -INFINITY) ? 0.f : z1 * ex2(m1 - n1);
+    m0 = n0;
+    m1 = n1;
+    const float s0 = (m0 == -INFINITY) ? 0.f : -m0, s1 = (m1 == -INFINITY) ? 0.f : -m1;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      z0 += ex2(c[nt][0] + s0) + ex2(c[nt][1] + s0);
+      z1 += ex2(c[nt][2] + s1) + ex2(c[nt][3] + s1);
     }
     __syncthreads();
   }
