@@ -3,15 +3,21 @@
 // MMInference ("key machinery"): block-sparse FlashAttention-style kernels load only the
 // permuted blocks and keep the tensor-core compute dense; "Grid-Shape Flash Attention"
 // (Algorithm 5) is the FlashAttention-2 online softmax over those blocks.  Here:
-//  - one persistent CTA per SM runs two independent streams of 128-query work items; each
-//    stream takes the next item from a global counter when it needs one (items are in
-//    plan order, most keys first, so the greedy assignment balances the SMs);
+//  - one persistent CTA per SM runs two independent streams of work units (a 128-query work
+//    item, or, for long sequences whose keys are cut into chunks, the item's tiles of one key
+//    chunk); each stream takes the next unit from a global counter when it needs one (plan
+//    order: grouped so that the units in flight share one head's K/V in L2, longest first);
+//  - a unit after its item's first key chunk resumes the item's online softmax from an
+//    accumulator in the workspace (unnormalised O, running max and sum), handed over between
+//    units through a per-item counter (release / acquire);
 //  - warps 0 and 2 stream the Q, K and V tiles of stream 0 and 1 with TMA (128-byte
 //    swizzle) into single-buffered slots of their own;
 //  - warps 1 and 3 (one thread each) issue the tcgen05.mma of stream 0 and 1:
 //    S_s = Q_s K^T into stream s's TMEM columns, then O_s += P_s V with P_s read from TMEM
-//    and O_s resident in TMEM for the whole work item.  While one stream's softmax runs, the
-//    tensor core works on the other stream;
+//    and O_s resident in TMEM for the whole unit; a group [PV(j), QK(j + 1)] is issued under
+//    a lock shared by the two issuers, so the tensor pipe receives whole groups back to back
+//    and the streams settle half a cycle apart: one stream's MMAs run while the other
+//    stream computes its softmax;
 //  - warps 4..7 (stream 0) and 8..11 (stream 1) each own TMEM lanes 0..127, one query row per
 //    thread and all 128 keys of every tile: they read S with tcgen05.ld, apply the element
 //    mask (causal in original positions + the head's pattern), run the online softmax in fp32
