@@ -249,6 +249,8 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {status} after warm-up")
     tiles, items = plan.tile_stats(ws)
     exec_flops = msa.executed_flops(tiles)
+    # allowed (query, key) pairs under the masks, counted on the device before the timed region
+    useful_flops = 4 * p.d * int(plan.mask_pairs(ws).sum())
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -371,8 +373,9 @@ def run_ours(args, rank, world, local_rank):
             "stages_ms": {"estimate": float(stage[:, 0].mean()), "permute": float(stage[:, 1].mean()),
                           "attention": attn_ms, "unpermute": float(stage[:, 3].mean())},
             "executed_tiles": tiles, "work_items": items, "executed_flops": exec_flops,
-            "dense_causal_flops": dense_causal_flops(p),
-            "dense_flops_avoided": dense_causal_flops(p) - exec_flops,
+            "useful_flops": useful_flops, "dense_causal_flops": dense_causal_flops(p),
+            "mask_density": useful_flops / dense_causal_flops(p),
+            "dense_flops_avoided": dense_causal_flops(p) - useful_flops,
             "attn_tflops": achieved,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": sm,
@@ -417,6 +420,7 @@ def run_sweep(args):
                     stages.append([ev[j].elapsed_time(ev[j + 1]) for j in range(4)])
             assert plan.device_status(ws) == 0
             tiles, _ = plan.tile_stats(ws)
+            useful = 4 * p.d * int(plan.mask_pairs(ws).sum())
             st_ms = np.mean(np.array(stages), axis=0)
             flops = msa.executed_flops(tiles)
             print(json.dumps({"sweep": "llama3-8b-text", "L": L, "budget": b, "warmup": warm, "steps": steps,
@@ -426,6 +430,7 @@ def run_sweep(args):
                               "estimate_over_attention": float(st_ms[0] / st_ms[2]),
                               "executed_flops": flops, "dense_causal_flops": dense_causal_flops(p),
                               "density": flops / dense_causal_flops(p),
+                              "mask_density": useful / dense_causal_flops(p),
                               "attn_tflops": flops / (st_ms[2] * 1e-3) / 1e12}), flush=True)
             del ws, plan
             torch.cuda.empty_cache()

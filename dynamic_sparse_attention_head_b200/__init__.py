@@ -73,6 +73,7 @@ def _load():
         "msa_read_tiles": ([_P, _P, _I32, _P, ctypes.POINTER(_I64), _P], _I32),
         "msa_tile_stats": ([_P, _P, _P, _P], _I32),
         "msa_attention_units": ([_P, _P], _I32),
+        "msa_mask_pairs": ([_P, _P, _P, _P], _I32),
         "msa_device_status": ([_P, _P, _P], _I32),
         "msa_status_string": ([_I32], ctypes.c_char_p),
         "msa_kernel_launches": ([], ctypes.c_uint64),
@@ -88,7 +89,7 @@ def _load():
 _lib = _load()
 EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_estimate", "msa_set_indices",
            "msa_permute", "msa_sparse_prefill", "msa_unpermute", "msa_read_indices", "msa_read_tiles",
-           "msa_tile_stats", "msa_attention_units", "msa_device_status", "msa_status_string",
+           "msa_tile_stats", "msa_attention_units", "msa_mask_pairs", "msa_device_status", "msa_status_string",
            "msa_kernel_launches", "msa_vslash_estimate_static")
 
 
@@ -313,6 +314,14 @@ class Plan:
         t = (_I64 * 2)()
         _check("msa_tile_stats", _lib.msa_tile_stats(self._h, ws.data_ptr(), ctypes.cast(t, _P), _stream_ptr(stream)))
         return int(t[0]), int(t[1])
+
+    def mask_pairs(self, ws, stream=None):
+        """Allowed (query, key) pairs per query head under the current masks (int64 [Hq]);
+        useful FLOPs = 4 * d * sum."""
+        import numpy as np
+        c = np.zeros(self.problem.Hq, np.int64)
+        _check("msa_mask_pairs", _lib.msa_mask_pairs(self._h, ws.data_ptr(), c.ctypes.data_as(_P), _stream_ptr(stream)))
+        return c
 
     def attention_units(self):
         """(work units, key chunks) of msa_sparse_prefill for this plan."""

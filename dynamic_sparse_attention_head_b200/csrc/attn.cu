@@ -302,6 +302,29 @@ __device__ __forceinline__ void mask_finish(const RowCtx& rc, const MaskRaw& r, 
   }
 }
 
+// Mask state of query row `t` of an item (row it.row0 + t of its class).
+__device__ __forceinline__ void fill_row_ctx(const AttnParams& p, const ItemInfo& it, const ClassStatic& cs, int t,
+                                             RowCtx& rc) {
+  const int r = it.row0 + t;
+  rc.valid = r < it.nrows;
+  const int32_t* rows = reinterpret_cast<const int32_t*>(p.ws + cs.rows_off);
+  rc.qpos = rc.valid ? ((cs.flags & CF_PERMUTED) ? __ldg(rows + r) : r) : 0;
+  rc.qcoord = (cs.flags & CF_RANK) ? r : rc.qpos;
+  rc.flags = cs.flags;
+  rc.sink = cs.sink;
+  rc.band = cs.band;
+  rc.kc_lo = cs.kc_lo;
+  rc.kc_hi = cs.kc_hi;
+  rc.krow_lo = cs.krow_lo;
+  rc.x_row0 = cs.x_row0;
+  rc.nwords = (p.L + 31) >> 5;
+  rc.blk_wpr = cs.blk_wpr;
+  rc.slash = reinterpret_cast<const uint32_t*>(p.ws + cs.slash_bits_off);
+  rc.excl = reinterpret_cast<const uint32_t*>(p.ws + cs.excl_bits_off);
+  rc.blk = reinterpret_cast<const uint32_t*>(p.ws + cs.blk_bits_off);
+  rc.xpos = reinterpret_cast<const int32_t*>(p.ws + cs.x_pos_off);
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -631,23 +654,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const ClassStatic& cs = class_of(p, it.cls);
       const int r = it.row0 + t;
       RowCtx& rc = sm.rctx[threadIdx.x - 128];
-      rc.valid = r < it.nrows;
-      const int32_t* rows = reinterpret_cast<const int32_t*>(p.ws + cs.rows_off);
-      rc.qpos = rc.valid ? ((cs.flags & CF_PERMUTED) ? __ldg(rows + r) : r) : 0;
-      rc.qcoord = (cs.flags & CF_RANK) ? r : rc.qpos;
-      rc.flags = cs.flags;
-      rc.sink = cs.sink;
-      rc.band = cs.band;
-      rc.kc_lo = cs.kc_lo;
-      rc.kc_hi = cs.kc_hi;
-      rc.krow_lo = cs.krow_lo;
-      rc.x_row0 = cs.x_row0;
-      rc.nwords = (p.L + 31) >> 5;
-      rc.blk_wpr = cs.blk_wpr;
-      rc.slash = reinterpret_cast<const uint32_t*>(p.ws + cs.slash_bits_off);
-      rc.excl = reinterpret_cast<const uint32_t*>(p.ws + cs.excl_bits_off);
-      rc.blk = reinterpret_cast<const uint32_t*>(p.ws + cs.blk_bits_off);
-      rc.xpos = reinterpret_cast<const int32_t*>(p.ws + cs.x_pos_off);
+      fill_row_ctx(p, it, cs, t, rc);
       const size_t orow = ((size_t)it.head * p.LP + it.qrow0 + r) * D;
 
       if (it.ntiles == 0) {
@@ -885,7 +892,55 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t heads, int
   return r == CUDA_SUCCESS;
 }
 
+// Allowed (query, key) pairs of every head: the attention kernel's element mask evaluated over
+// each work item's whole tile list (one thread per query row), full tiles counted as 128 per
+// valid row, summed per head.  Keys that a gathered tile serves are excluded from the identity
+// tiles, so every pair is counted once.
+__global__ void __launch_bounds__(TILE) mask_count_kernel(const AttnParams p, unsigned long long* counts) {
+  const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+    ItemInfo it;
+    if (!load_item(p, item, it)) continue;
+    RowCtx rc;
+    fill_row_ctx(p, it, class_of(p, it.cls), threadIdx.x, rc);
+    unsigned long long n = 0;
+    for (int tt = 0; tt < it.ntiles; ++tt) {
+      const uint32_t tile = __ldg(tiles + it.tile0 + tt);
+      if (tile & TILE_FULL) {
+        n += rc.valid ? TILE : 0;
+        continue;
+      }
+      MaskRaw raw;
+      uint32_t mk[4];
+      mask_prefetch(rc, tile, raw);
+      mask_finish(rc, raw, mk);
+      n += __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_down_sync(0xFFFFFFFFu, n, o);
+    if ((threadIdx.x & 31) == 0 && n) atomicAdd(counts + it.head, n);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_mask_count(const DevPlan& dp, cudaStream_t st) {
+  AttnParams p{};
+  p.ws = dp.ws;
+  p.lay = dp.lay;
+  p.L = (int32_t)dp.L;
+  p.Hq = dp.Hq;
+  p.Hkv = dp.Hkv;
+  p.LP = dp.LP;
+  p.n_items = dp.n_items;
+  auto* counts = reinterpret_cast<unsigned long long*>(const_cast<uint8_t*>(dp.ws + dp.lay.mask_pairs));
+  if (cudaError_t e = cudaMemsetAsync(counts, 0, 8 * (size_t)dp.Hq, st)) return e;
+  if (dp.n_items == 0) return cudaSuccess;
+  const int grid = std::max(1, std::min(dp.n_items, sm_count() * 8));
+  count_launches(1);
+  mask_count_kernel<<<grid, TILE, 0, st>>>(p, counts);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
                              float* lse, cudaStream_t st) {

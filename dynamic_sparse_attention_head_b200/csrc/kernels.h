@@ -55,5 +55,7 @@ cudaError_t launch_unpermute(const DevPlan& dp, void* O, const msa_strides& s, c
 // attention
 cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
                              float* lse, cudaStream_t st);
+// allowed (query, key) pairs per head over the tile lists, into the workspace's mask_pairs
+cudaError_t launch_mask_count(const DevPlan& dp, cudaStream_t st);
 
 }  // namespace msa

@@ -160,6 +160,7 @@ struct Layout {
   int64_t chunk_done;        // uint32 [n_items]: chunks of the item whose state is in its accumulator
   int64_t acc;               // fp32 [n_acc][128][ACC_ROW]: per-item online-softmax state between chunks
   int64_t tiles;             // uint32 [total tile capacity]: (src << 28) | TILE_FULL? | first key row
+  int64_t mask_pairs;        // uint64 [Hq]: allowed (query, key) pairs per head (msa_mask_pairs)
   int64_t modality;          // uint8 [L]
   int64_t rank;              // int32 [L]
   int64_t perm2d;            // int32 [L] modality-grouped order (text then video) -> position

@@ -480,6 +480,7 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
     lay.acc = B.take(4 * 2 * (int64_t)P->band_cap * TILE * ACC_ROW, 1024);
   }
   lay.tiles = B.take(4 * P->total_tiles);
+  lay.mask_pairs = B.take(8 * (int64_t)Hq);
   lay.modality = B.take(L);
   lay.rank = B.take(4 * L);
   lay.perm2d = B.take(4 * L);
@@ -889,6 +890,20 @@ msa_status msa_tile_stats(const msa_plan* P, const void* ws, int64_t tiles[2], v
   }
   tiles[0] = t;
   tiles[1] = n;
+  return MSA_OK;
+}
+
+msa_status msa_mask_pairs(const msa_plan* P, void* ws, int64_t* counts, void* stream) {
+  if (!P || !ws || !counts) return MSA_ERR_INVALID_ARG;
+  if (P->ready_ws != ws) return MSA_ERR_STATE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaError_t e = launch_mask_count(dev(P, ws), cs)) return cuda_status(e);
+  std::vector<uint64_t> c(P->Hq);
+  if (cudaMemcpyAsync(c.data(), static_cast<const uint8_t*>(ws) + P->lay.mask_pairs, 8 * c.size(),
+                      cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return MSA_ERR_CUDA;
+  for (int32_t h = 0; h < P->Hq; ++h) counts[h] = (int64_t)c[h];
   return MSA_OK;
 }
 

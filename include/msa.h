@@ -191,6 +191,16 @@ msa_status msa_read_indices(const msa_plan* plan, const void* ws, int32_t head, 
  * Executed block FLOPs = 4 * 128 * 128 * 128 * tiles[0]. */
 msa_status msa_tile_stats(const msa_plan* plan, const void* ws, int64_t tiles[2], void* stream);
 
+/* Allowed (query, key) pairs of each query head under the masks of the last msa_estimate /
+ * msa_set_indices in this workspace: causal in original positions and the head's pattern, each
+ * pair once (MInference / MMInference: the token-level masks of the A-shape, vertical-slash,
+ * block-sparse, grid, Q-boundary and 2D-boundary heads).  counts: host int64 [Hq].  Useful
+ * FLOPs = 4 * d * sum(counts); the executed block FLOPs of msa_tile_stats also count the masked
+ * entries of the executed tiles.  Runs a counting kernel over the tile lists with the attention
+ * kernel's mask logic on `stream` and synchronises it; MSA_ERR_STATE if the workspace holds no
+ * indices of this plan. */
+msa_status msa_mask_pairs(const msa_plan* plan, void* ws, int64_t* counts, void* stream);
+
 /* How msa_sparse_prefill divides its work (host only, no device access): out[0] = work units,
  * out[1] = key chunks.  When one head's K and V exceed about 96 MB (L > 192K tokens) the keys
  * are cut into chunks of 65536 (the environment variable MSA_ATTN_CHUNK_KEYS, a multiple of

@@ -86,6 +86,23 @@ def test_tiles_cover_mask_exactly_once(name):
             assert n_full > 0, f"{name} head {h}: no tile flagged full"
 
 
+@pytest.mark.parametrize("name", list(PROBLEMS) + ["mixed"])
+def test_mask_pairs_match_oracle(name):
+    """Allowed pairs per head counted on the device with the kernel's mask logic equal the
+    oracle's token-level mask counts exactly (the useful FLOPs the bench reports)."""
+    p = mixed_problem() if name == "mixed" else PROBLEMS[name]
+    Q, K, V = make_inputs(p, seed=5)
+    idx = oracle.estimate(p, Q, K)
+    plan, ws, _, _ = _run(p, Q, K, V, idx)
+    got = plan.mask_pairs(ws)
+    ref = np.array([int(oracle.mask_count(p, h, idx[h]).sum()) for h in range(p.Hq)], np.int64)
+    assert np.array_equal(got, ref), f"{name}: device {got.tolist()} oracle {ref.tolist()}"
+    if name == "dense":
+        assert np.all(got == p.L * (p.L + 1) // 2)
+    tiles, _ = plan.tile_stats(ws)
+    assert got.sum() <= tiles * 128 * 128
+
+
 def test_dense_executes_causal_tiles_only():
     p = PROBLEMS["dense"]
     Q, K, V = make_inputs(p, seed=3)

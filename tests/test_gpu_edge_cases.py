@@ -35,6 +35,9 @@ def _forward(p, Q, K, V, q=None, k=None, v=None, o=None):
     torch.cuda.synchronize()
     assert plan.device_status(ws) == 0
     idx = [plan.read_indices(h, ws) for h in range(p.Hq)]
+    # allowed pairs per head under the device's index sets: exact against the oracle's masks
+    ref = [int(oracle.mask_count(p, h, idx[h]).sum()) for h in range(p.Hq)]
+    assert plan.mask_pairs(ws).tolist() == ref, f"{p.name}: mask pair counts"
     return idx, o, lse.cpu().numpy()
 
 
