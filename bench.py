@@ -484,8 +484,6 @@ def executed_flops_for(p, per_kind):
     except Exception:
         return None
     idx = [per_kind[h.kind]["idx"] for h in p.heads]
-    if any(h.kind == "block" for h in p.heads):
-        pass
     plan = msa.Plan(p)
     ws = plan.alloc_workspace()
     plan.set_indices(idx, ws)

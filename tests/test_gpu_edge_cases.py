@@ -109,3 +109,20 @@ def test_single_modality_layout(modality):
     Q, K, V = make_inputs(p, seed=9)
     idx, o, lse = _forward(p, Q, K, V)
     _check(p, Q, K, V, idx, o, lse, p.name)
+
+
+def test_calls_out_of_order_are_refused():
+    """Permute, prefill and the mask count need this plan's indices in the workspace first."""
+    p = Problem(L=256, Hq=1, Hkv=1, segments=[(0, 256, TEXT)], heads=[Head("vslash", k_v=4, k_s=8)],
+                name="order")
+    Q, K, V = make_inputs(p, seed=9)
+    plan = msa.Plan(p)
+    ws = plan.alloc_workspace()
+    q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+    for call in (lambda: plan.mask_pairs(ws), lambda: plan.permute(q, k, v, ws),
+                 lambda: plan.sparse_prefill(q, k, v, ws)):
+        with pytest.raises(msa.MsaError) as e:
+            call()
+        assert e.value.code == 9  # MSA_ERR_STATE
+    plan.estimate(q, k, ws)
+    assert plan.mask_pairs(ws).shape == (1,)
