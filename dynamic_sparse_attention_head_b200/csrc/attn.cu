@@ -983,11 +983,13 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
     if (cudaError_t e = cudaMemsetAsync(p.chunk_done, 0, sizeof(uint32_t) * (size_t)dp.n_items, st)) return e;
   }
   const size_t smem = sizeof(AttnSmem);
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev)) return e;
+  if (device_pending(configured, dev)) {
     cudaError_t e = cudaFuncSetAttribute(msa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    configured = true;
+    mark_device(configured, dev);
   }
   const int grid = std::max(1, std::min((dp.n_units + N_STREAMS - 1) / N_STREAMS, sm_count()));
   count_launches(1);

@@ -648,11 +648,15 @@ cudaError_t launch_lastq(const DevPlan& dp, const void* Q, const void* K, const 
   if (dp.has2d && (e = launch_group_k(dp, K, s, st)) != cudaSuccess) return e;
   const size_t smem1 = sizeof(LqSmem);
   const size_t smem2 = sizeof(LqSmem) + sizeof(float) * SACC_MAX;
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(lastq_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-    cudaFuncSetAttribute(lastq_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
-    configured = true;
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (device_pending(configured, dev)) {
+    if ((e = cudaFuncSetAttribute(lastq_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(lastq_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) != cudaSuccess)
+      return e;
+    mark_device(configured, dev);
   }
   if (dp.sacc_n < 0 || dp.sacc_n > SACC_MAX) return cudaErrorInvalidValue;
   const size_t smem2_used = sizeof(LqSmem) + sizeof(float) * (size_t)dp.sacc_n;

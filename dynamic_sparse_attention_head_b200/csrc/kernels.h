@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "msa_internal.h"
 
 namespace msa {
@@ -31,7 +33,16 @@ struct DevPlan {
   const int32_t* class_kind;  // host copy: kind of each class
 };
 
-int sm_count();
+int sm_count();  // SMs of the current device
+
+// One-time setup per device (function attributes such as the dynamic shared-memory limit are
+// per device): pending until marked for device `dev`.
+inline bool device_pending(const std::atomic<uint64_t>& flags, int dev) {
+  return dev < 0 || dev >= 64 || !((flags.load(std::memory_order_acquire) >> dev) & 1u);
+}
+inline void mark_device(std::atomic<uint64_t>& flags, int dev) {
+  if (dev >= 0 && dev < 64) flags.fetch_or(1ull << dev, std::memory_order_release);
+}
 // bumps the library-wide kernel launch counter by n
 void count_launches(int n);
 
