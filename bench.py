@@ -216,10 +216,31 @@ def run_ours(args, rank, world, local_rank):
     q, k, v = dev_copy(Qh), dev_copy(Kh), dev_copy(Vh)
     o = torch.empty_like(q)
     plan = msa.Plan(p)
-    ws = plan.alloc_workspace()
+    ws = plan.alloc_workspace(indexed=args.indexed)
     stream = torch.cuda.current_stream()
 
     n_steps = [0]
+
+    def prefill(bq, bk, bv, bo, events=None):
+        """permute -> sparse prefill -> unpermute, or the one index-based call (--indexed; the
+        permute and unpermute stages are then empty and the key gathers run inside the call)."""
+        if args.indexed:
+            if events is not None:
+                events[2].record(stream)
+            plan.sparse_prefill_indexed(bq, bk, bv, ws, bo)
+            if events is not None:
+                events[3].record(stream)
+                events[4].record(stream)
+            return
+        plan.permute(bq, bk, bv, ws)
+        if events is not None:
+            events[2].record(stream)
+        plan.sparse_prefill(bq, bk, bv, ws)
+        if events is not None:
+            events[3].record(stream)
+        plan.unpermute(ws, bo)
+        if events is not None:
+            events[4].record(stream)
 
     def step(events=None):
         if events is not None:
@@ -231,15 +252,7 @@ def run_ours(args, rank, world, local_rank):
         n_steps[0] += 1
         if events is not None:
             events[1].record(stream)
-        plan.permute(q, k, v, ws)
-        if events is not None:
-            events[2].record(stream)
-        plan.sparse_prefill(q, k, v, ws)
-        if events is not None:
-            events[3].record(stream)
-        plan.unpermute(ws, o)
-        if events is not None:
-            events[4].record(stream)
+        prefill(q, k, v, o, events)
 
     for _ in range(args.warmup):
         step()
@@ -310,9 +323,7 @@ def run_ours(args, rank, world, local_rank):
                 if s_ >= 2:
                     stream.wait_event(out_done[b])  # O of step s-2 has reached the host
                 plan.estimate(bq, bk, ws)
-                plan.permute(bq, bk, bv, ws)
-                plan.sparse_prefill(bq, bk, bv, ws)
-                plan.unpermute(ws, bo)
+                prefill(bq, bk, bv, bo)
                 comp_done[b].record(stream)
                 with torch.cuda.stream(d2h):
                     d2h.wait_event(comp_done[b])
@@ -342,12 +353,14 @@ def run_ours(args, rank, world, local_rank):
     achieved = exec_flops / (attn_ms * 1e-3) / 1e12
     peak_sus = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    traffic = recorded_traffic(args.workload)
+    traffic = recorded_traffic(args.workload + ("+indexed" if args.indexed else ""))
     roofline = {"kernel": "msa_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": peak_sus,
                 "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
                 "peak_source": f"{pk_src} bf16_tflops_sustained (kernel inside a long step)",
                 "frac_of_burst_peak": achieved / peak_burst,
-                "flops_per_launch": exec_flops, "ms_per_launch": attn_ms}
+                "flops_per_launch": exec_flops, "ms_per_launch": attn_ms,
+                **({"timed": "msa_sparse_prefill_indexed: the key gathers (a few % of its bytes, "
+                             "under 0.2 % of its time) and the attention kernel"} if args.indexed else {})}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -369,7 +382,9 @@ def run_ours(args, rank, world, local_rank):
             "config": {"workload": args.workload, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
                        "heads": kind_summary(p), "parallelism": f"independent layer per rank x{world}",
                        "l2": "inputs larger than L2 (no flush)" if (Qh.nbytes > 126e6) else "inputs smaller than L2",
-                       "seed": "rank", **({"estimate_every": args.estimate_every} if args.estimate_every > 1 else {})},
+                       "seed": "rank", **({"estimate_every": args.estimate_every} if args.estimate_every > 1 else {}),
+                       **({"path": "index-based (Q rows gathered in the attention kernel, O written at "
+                                   "original positions)"} if args.indexed else {})},
             "stages_ms": {"estimate": float(stage[:, 0].mean()), "permute": float(stage[:, 1].mean()),
                           "attention": attn_ms, "unpermute": float(stage[:, 3].mean())},
             "executed_tiles": tiles, "work_items": items, "executed_flops": exec_flops,
@@ -505,6 +520,9 @@ def main():
     ap.add_argument("--estimate-every", type=int, default=1,
                     help="estimate indices on every K-th layer only and reuse them in between (index "
                          "amortisation across layers of one layout; 1, the default, is the benchmark)")
+    ap.add_argument("--indexed", action="store_true",
+                    help="index-based prefill (msa_sparse_prefill_indexed) in place of permute -> "
+                         "sparse prefill -> unpermute")
     ap.add_argument("--sweep-lengths", default=",".join(str(x) for x in workload.SWEEP_LENGTHS))
     ap.add_argument("--sweep-budgets", default="0.02,0.05,0.1,0.25,dense")
     args = ap.parse_args()

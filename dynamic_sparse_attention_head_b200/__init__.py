@@ -64,6 +64,9 @@ def _load():
         "msa_plan_create": ([ctypes.POINTER(ProblemC), ctypes.POINTER(_P)], _I32),
         "msa_plan_destroy": ([_P], None),
         "msa_workspace_bytes": ([_P], ctypes.c_size_t),
+        "msa_workspace_bytes_indexed": ([_P], ctypes.c_size_t),
+        "msa_sparse_prefill_indexed": ([_P, _P, _P, _P, _P, ctypes.POINTER(Strides), _P, ctypes.c_size_t, _P, _P],
+                                       _I32),
         "msa_estimate": ([_P, _P, _P, ctypes.POINTER(Strides), _P, ctypes.c_size_t, _P], _I32),
         "msa_set_indices": ([_P, _P, _P, ctypes.c_size_t, _P], _I32),
         "msa_permute": ([_P, _P, _P, _P, ctypes.POINTER(Strides), _P, ctypes.c_size_t, _P], _I32),
@@ -87,7 +90,8 @@ def _load():
 
 
 _lib = _load()
-EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_estimate", "msa_set_indices",
+EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_workspace_bytes_indexed",
+           "msa_sparse_prefill_indexed", "msa_estimate", "msa_set_indices",
            "msa_permute", "msa_sparse_prefill", "msa_unpermute", "msa_read_indices", "msa_read_tiles",
            "msa_tile_stats", "msa_attention_units", "msa_mask_pairs", "msa_device_status", "msa_status_string",
            "msa_kernel_launches", "msa_vslash_estimate_static")
@@ -157,15 +161,19 @@ class Plan:
         _check("msa_plan_create", _lib.msa_plan_create(ctypes.byref(pc), ctypes.byref(h)))
         self._h = h
         self.workspace_bytes = int(_lib.msa_workspace_bytes(h))
+        self.workspace_bytes_indexed = int(_lib.msa_workspace_bytes_indexed(h))
 
     def __del__(self):
         if getattr(self, "_h", None):
             _lib.msa_plan_destroy(self._h)
             self._h = None
 
-    def alloc_workspace(self):
+    def alloc_workspace(self, indexed: bool = False):
+        """Device workspace for the three-call path, or (indexed) the smaller one of the
+        index-based path."""
         import torch
-        return torch.empty(self.workspace_bytes, dtype=torch.uint8, device="cuda")
+        n = self.workspace_bytes_indexed if indexed else self.workspace_bytes
+        return torch.empty(n, dtype=torch.uint8, device="cuda")
 
     # ---- the four steps --------------------------------------------------------------
     def estimate(self, Q, K, ws, stream=None):
@@ -229,9 +237,22 @@ class Plan:
         _check("msa_unpermute", _lib.msa_unpermute(self._h, ws.data_ptr(), ws.numel(), O.data_ptr(), ctypes.byref(s),
                                                    _stream_ptr(stream)))
 
-    def forward(self, Q, K, V, ws, O, lse=None, stream=None):
-        """The whole path: estimate -> permute -> sparse prefill -> unpermute."""
+    def sparse_prefill_indexed(self, Q, K, V, ws, O, lse=None, stream=None):
+        """Permute + sparse prefill + unpermute in one call: Q rows gathered by index in the
+        kernel, O written at original positions."""
+        s = _strides(Q=Q, K=K, V=V, O=O)
+        _check("msa_sparse_prefill_indexed",
+               _lib.msa_sparse_prefill_indexed(self._h, Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(),
+                                               ctypes.byref(s), ws.data_ptr(), ws.numel(),
+                                               lse.data_ptr() if lse is not None else None, _stream_ptr(stream)))
+
+    def forward(self, Q, K, V, ws, O, lse=None, stream=None, indexed: bool = False):
+        """The whole path: estimate -> permute -> sparse prefill -> unpermute, or (indexed)
+        estimate -> index-based sparse prefill."""
         self.estimate(Q, K, ws, stream)
+        if indexed:
+            self.sparse_prefill_indexed(Q, K, V, ws, O, lse, stream)
+            return
         self.permute(Q, K, V, ws, stream)
         self.sparse_prefill(Q, K, V, ws, lse, stream)
         self.unpermute(ws, O, stream)

@@ -50,6 +50,13 @@ struct AttnParams {
   int32_t n_units, n_kchunks, n_bands;
   uint32_t* chunk_done;    // per item: chunks whose state is in its accumulator (chunked keys)
   float* acc;              // accumulator slots [slot][128][ACC_ROW] (chunked keys)
+  // index-based prefill (od not null): the Q rows of permuted classes are gathered from the
+  // caller's Q by row index, and every output row goes to the caller's O at its original
+  // position; otherwise Q comes from the permuted copy and O goes to the permuted O copy
+  const __nv_bfloat16* qg;
+  int64_t qg_head, qg_row;
+  __nv_bfloat16* od;
+  int64_t od_head, od_row;
 };
 
 // warpgroup 0: warps 0 / 2 TMA of stream 0 / 1, warps 1 / 3 MMA of stream 0 / 1; warpgroups
@@ -83,6 +90,7 @@ struct __align__(1024) AttnSmem {
   uint64_t q_full[N_STREAMS], q_empty[N_STREAMS];
   uint64_t k_full[N_STREAMS], k_empty[N_STREAMS];
   uint64_t v_full[N_STREAMS], v_empty[N_STREAMS];
+  uint64_t qg_full[N_STREAMS];  // Q gathered by the softmax warpgroup (index-based prefill)
   uint64_t s_full[N_STREAMS], p_full[N_STREAMS];
   uint64_t o_full[N_STREAMS], o_free[N_STREAMS];
   // work-item queue of each stream: ids taken from the global counter by the stream's TMA
@@ -396,12 +404,13 @@ __device__ __forceinline__ void issue_unlock(int* lock) { atomicExch(lock, 0); }
 // stream whose group follows the other's gets its S one group later and starts its softmax
 // then: the streams settle half a cycle apart, and one stream's MMAs run while the other
 // computes its softmax.
+template <bool INDEXED>
 __device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, uint32_t tmem, int s,
                                            volatile int* abort) {
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
   const uint32_t s_col = tmem + TM_STREAM * s;
-  uint32_t q_use = 0, k_use = 0, v_use = 0, done = 0;
+  uint32_t q_use = 0, qg_use = 0, k_use = 0, v_use = 0, done = 0;
   auto qk = [&](bool last) {
     tc_fence_after();
     uint32_t q_addr = smem_addr(sm.q[s]), k_addr = smem_addr(sm.k[s]);
@@ -429,8 +438,13 @@ __device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, ui
     if (!load_unit(p, e, it, un) || it.ntiles == 0) continue;
     const int n = it.ntiles;
     const bool cont = un.k > 0;  // O starts from the item's accumulator (loaded by the softmax)
-    if (!mbar_wait(&sm.q_full[s], q_use & 1, abort)) return;
-    ++q_use;
+    if (INDEXED && it.q_src) {  // Q gathered by index by the softmax warpgroup
+      if (!mbar_wait(&sm.qg_full[s], qg_use & 1, abort)) return;
+      ++qg_use;
+    } else {
+      if (!mbar_wait(&sm.q_full[s], q_use & 1, abort)) return;
+      ++q_use;
+    }
     if (!mbar_wait(&sm.k_full[s], k_use & 1, abort)) return;
     if (!issue_lock(&sm.issue_lock, abort)) return;
     qk(n == 1);
@@ -460,6 +474,10 @@ __device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, ui
   }
 }
 
+// INDEXED: the index-based prefill (Q rows of permuted classes gathered by row index, output
+// rows written at their original positions), compiled separately so that the other path keeps
+// its code unchanged.
+template <bool INDEXED>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     msa_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQp,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -487,6 +505,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
+      mbar_init(&sm.qg_full[s], 128);
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 128);
       mbar_init(&sm.o_full[s], 1);
@@ -558,7 +577,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         if (qk_live && qk_op >= 0) {
           if (qk_op == 0) {
-            if (q_iss == 0 || mbar_test(&sm.q_empty[s], (q_iss - 1) & 1)) {
+            if (INDEXED && qk_it.q_src) {  // gathered by the softmax warpgroup; q_empty still
+              ++q_iss;                  // completes once per item
+              qk_op = 1;
+              wd.progress();
+            } else if (q_iss == 0 || mbar_test(&sm.q_empty[s], (q_iss - 1) & 1)) {
               mbar_arrive_expect_tx(&sm.q_full[s], TILE_BYTES);
               if (qk_it.q_src) {
                 tma_load_3d(sm.q[s], &tmQp, &sm.q_full[s], 0, qk_it.qrow0 + qk_it.row0, qk_it.q_slice);
@@ -623,7 +646,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // ------------------------------------------------------------------ MMA issuers
     // warp 1: stream 0, warp 3: stream 1
     if (lane == 0) {
-      mma_stream(p, sm, tmem, warp >> 1, abort);
+      mma_stream<INDEXED>(p, sm, tmem, warp >> 1, abort);
       // wait for every MMA issued by this thread before the tensor memory is released
       umma_commit(&sm.drain[warp >> 1]);
       mbar_wait(&sm.drain[warp >> 1], 0, abort, 100000000ull);
@@ -657,9 +680,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       fill_row_ctx(p, it, cs, t, rc);
       const size_t orow = ((size_t)it.head * p.LP + it.qrow0 + r) * D;
 
+      // the unit's output row: the caller's O at the original position (index-based), or the
+      // permuted O copy
+      auto out_row = [&]() -> uint4* {
+        return reinterpret_cast<uint4*>(INDEXED ? p.od + (size_t)it.head * p.od_head + (size_t)rc.qpos * p.od_row
+                                                : op + orow);
+      };
       if (it.ntiles == 0) {
         if (rc.valid) {
-          uint4* dst = reinterpret_cast<uint4*>(op + orow);
+          uint4* dst = out_row();
 #pragma unroll
           for (int i = 0; i < 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
           if (p.lse) p.lse[(size_t)it.head * p.L + rc.qpos] = -INFINITY;
@@ -667,6 +696,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         continue;
       }
 
+      if (INDEXED && it.q_src) {
+        // Q row t of the unit from the caller's Q at its original position (zeros for rows past
+        // the class) into the stream's Q slot in the 128-byte-swizzled layout the MMA reads:
+        // 16-byte chunk c of row t at chunk c ^ (t & 7).  The slot is free: this warpgroup has
+        // read the S of the stream's previous unit, so its last QK is complete.
+        const __nv_bfloat16* src = p.qg + (size_t)it.head * p.qg_head + (size_t)rc.qpos * p.qg_row;
+        const uint32_t bytes = rc.valid ? 16u : 0u;
+        const uint32_t dst = smem_addr(sm.q[s]) + (uint32_t)t * 128u;
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            cp_async16_zfill(dst + a * ATOM_BYTES + ((uint32_t)(c ^ (t & 7)) << 4), src + a * 64 + c * 8, bytes);
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.qg_full[s]);
+      }
       float m_used = -INFINITY, l = 0.f;
       // A unit after the item's first key chunk resumes from the item's accumulator: the
       // previous chunk's unit releases it (chunk_done) once every row is stored.
@@ -826,7 +872,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         continue;
       }
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(op + orow);
+      uint4* dst = out_row();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t oa[32];
@@ -943,12 +989,13 @@ cudaError_t launch_mask_count(const DevPlan& dp, cudaStream_t st) {
 }
 
 cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
-                             float* lse, cudaStream_t st) {
+                             float* lse, void* O, cudaStream_t st) {
   CUtensorMap mq, mqp, mk, mv, mk2, mv2, mxk, mxv;
   const uint8_t* ws = dp.ws;
   bool ok = make_map(&mq, Q, dp.L, dp.Hq, s.q_row, s.q_head) && make_map(&mk, K, dp.L, dp.Hkv, s.k_row, s.k_head) &&
             make_map(&mv, V, dp.L, dp.Hkv, s.v_row, s.v_head) &&
-            make_map(&mqp, ws + dp.lay.qp, dp.LP, std::max(dp.n_qslices, 1), D, (int64_t)dp.LP * D) &&
+            (O ? make_map(&mqp, Q, dp.L, dp.Hq, s.q_row, s.q_head)  // unused: Q rows are gathered
+               : make_map(&mqp, ws + dp.lay.qp, dp.LP, std::max(dp.n_qslices, 1), D, (int64_t)dp.LP * D)) &&
             make_map(&mxk, ws + dp.lay.xk, dp.x_rows, std::max(dp.n_xslices, 1), D, (int64_t)dp.x_rows * D) &&
             make_map(&mxv, ws + dp.lay.xv, dp.x_rows, std::max(dp.n_xslices, 1), D, (int64_t)dp.x_rows * D);
   if (ok && dp.has2d) {
@@ -977,6 +1024,12 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
   p.n_bands = dp.n_bands;
   p.chunk_done = nullptr;
   p.acc = nullptr;
+  p.qg = static_cast<const __nv_bfloat16*>(Q);
+  p.qg_head = s.q_head;
+  p.qg_row = s.q_row;
+  p.od = static_cast<__nv_bfloat16*>(O);
+  p.od_head = s.o_head;
+  p.od_row = s.o_row;
   if (dp.n_kchunks > 1) {
     p.chunk_done = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(ws + dp.lay.chunk_done));
     p.acc = reinterpret_cast<float*>(const_cast<uint8_t*>(ws + dp.lay.acc));
@@ -987,13 +1040,18 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
   int dev = 0;
   if (cudaError_t e = cudaGetDevice(&dev)) return e;
   if (device_pending(configured, dev)) {
-    cudaError_t e = cudaFuncSetAttribute(msa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(msa_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(msa_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     mark_device(configured, dev);
   }
   const int grid = std::max(1, std::min((dp.n_units + N_STREAMS - 1) / N_STREAMS, sm_count()));
   count_launches(1);
-  msa_attn_kernel<<<grid, ATT_THREADS, smem, st>>>(mq, mqp, mk, mv, mk2, mv2, mxk, mxv, p);
+  if (O)
+    msa_attn_kernel<true><<<grid, ATT_THREADS, smem, st>>>(mq, mqp, mk, mv, mk2, mv2, mxk, mxv, p);
+  else
+    msa_attn_kernel<false><<<grid, ATT_THREADS, smem, st>>>(mq, mqp, mk, mv, mk2, mv2, mxk, mxv, p);
   return cudaGetLastError();
 }
 

@@ -60,12 +60,16 @@ cudaError_t launch_grid_detect(const DevPlan& dp, cudaStream_t st);
 cudaError_t launch_materialize(const DevPlan& dp, cudaStream_t st);
 cudaError_t launch_tiles(const DevPlan& dp, cudaStream_t st);
 // gathers
+// with_q: also the permuted Q copy (the index-based prefill gathers Q rows itself)
 cudaError_t launch_permute(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
-                           cudaStream_t st);
+                           bool with_q, cudaStream_t st);
 cudaError_t launch_unpermute(const DevPlan& dp, void* O, const msa_strides& s, cudaStream_t st);
 // attention
+// O null: the output goes to the permuted O copy in the workspace (msa_unpermute scatters it);
+// otherwise the Q rows of permuted classes are gathered by index and every output row is
+// written to O at its original position.
 cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
-                             float* lse, cudaStream_t st);
+                             float* lse, void* O, cudaStream_t st);
 // allowed (query, key) pairs per head over the tile lists, into the workspace's mask_pairs
 cudaError_t launch_mask_count(const DevPlan& dp, cudaStream_t st);
 

@@ -170,6 +170,7 @@ struct Layout {
   int64_t op;                // bf16 [n_qslices][q_rows][128] permuted O (+ identity heads)
   int64_t xk, xv;            // bf16 [n_xslices][x_rows][128] gathered K / V
   int64_t k2d, v2d;          // bf16 [Hkv][L][128] modality-grouped K / V
+  int64_t indexed_total;     // bytes msa_sparse_prefill_indexed uses: every region before qp
   int64_t total;
 };
 

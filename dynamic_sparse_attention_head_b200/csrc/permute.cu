@@ -116,12 +116,12 @@ __global__ void unpermute_kernel(DevPlan dp, __nv_bfloat16* O, int64_t oh, int64
 }  // namespace
 
 cudaError_t launch_permute(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
-                           cudaStream_t st) {
+                           bool with_q, cudaStream_t st) {
   const int bx = std::max(1, sm_count() * 4 / std::max(1, dp.Hq)) ;
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
   const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K);
   const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(V);
-  if (dp.n_qslices > 0) {
+  if (with_q && dp.n_qslices > 0) {
     count_launches(1);
     permute_q_kernel<<<dim3(bx * 2, dp.Hq), 256, 0, st>>>(dp, q, s.q_head, s.q_row);
   }

@@ -604,12 +604,14 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
     return MSA_ERR_INVALID_ARG;
   }
   lay.kbar = has_block ? B.take(4 * (int64_t)Hkv * nb * D) : 0;
-  lay.qp = B.take(2 * (int64_t)std::max(n_qslices, 1) * LP * D, 1024);
-  lay.op = B.take(2 * (int64_t)Hq * LP * D, 1024);
   lay.xk = B.take(2 * (int64_t)std::max(n_xslices, 1) * std::max(x_rows_max, TILE) * D, 1024);
   lay.xv = B.take(2 * (int64_t)std::max(n_xslices, 1) * std::max(x_rows_max, TILE) * D, 1024);
   lay.k2d = has2d ? B.take(2 * (int64_t)Hkv * L * D, 1024) : 0;
   lay.v2d = has2d ? B.take(2 * (int64_t)Hkv * L * D, 1024) : 0;
+  lay.indexed_total = round_up(B.off, 256);
+  // the permuted Q and O copies come last: the index-based prefill does without them
+  lay.qp = B.take(2 * (int64_t)std::max(n_qslices, 1) * LP * D, 1024);
+  lay.op = B.take(2 * (int64_t)Hq * LP * D, 1024);
   lay.total = round_up(B.off, 256);
 
   // ---- the blob uploaded into the workspace at every estimate / set_indices
@@ -669,6 +671,8 @@ void msa_plan_destroy(msa_plan* plan) { delete plan; }
 
 size_t msa_workspace_bytes(const msa_plan* plan) { return plan ? (size_t)plan->lay.total : 0; }
 
+size_t msa_workspace_bytes_indexed(const msa_plan* plan) { return plan ? (size_t)plan->lay.indexed_total : 0; }
+
 }  // extern "C"
 
 // ------------------------------------------------------------------------------------------
@@ -676,10 +680,12 @@ namespace {
 
 msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
-msa_status check_ws(const msa_plan* P, const void* ws, size_t bytes) {
+// `full`: the call uses the permuted Q / O copies (msa_permute, msa_sparse_prefill,
+// msa_unpermute); the others need only the indexed part of the layout.
+msa_status check_ws(const msa_plan* P, const void* ws, size_t bytes, bool full) {
   if (!P || !ws) return MSA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(ws) % 256) return MSA_ERR_ALIGN;
-  if (bytes < (size_t)P->lay.total) return MSA_ERR_WORKSPACE;
+  if (bytes < (size_t)(full ? P->lay.total : P->lay.indexed_total)) return MSA_ERR_WORKSPACE;
   return MSA_OK;
 }
 
@@ -707,7 +713,7 @@ extern "C" {
 
 msa_status msa_estimate(msa_plan* P, const void* Q, const void* K, const msa_strides* s, void* ws, size_t ws_bytes,
                         void* stream) {
-  msa_status st = check_ws(P, ws, ws_bytes);
+  msa_status st = check_ws(P, ws, ws_bytes, false);
   if (st != MSA_OK) return st;
   if (!s) return MSA_ERR_INVALID_ARG;
   if ((st = check_tensor(Q, s->q_head, s->q_row)) != MSA_OK) return st;
@@ -728,7 +734,7 @@ msa_status msa_estimate(msa_plan* P, const void* Q, const void* K, const msa_str
 }
 
 msa_status msa_set_indices(msa_plan* P, const msa_head_indices* heads, void* ws, size_t ws_bytes, void* stream) {
-  msa_status st = check_ws(P, ws, ws_bytes);
+  msa_status st = check_ws(P, ws, ws_bytes, false);
   if (st != MSA_OK) return st;
   if (!heads) return MSA_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -818,19 +824,19 @@ msa_status msa_set_indices(msa_plan* P, const msa_head_indices* heads, void* ws,
 
 msa_status msa_permute(msa_plan* P, const void* Q, const void* K, const void* V, const msa_strides* s, void* ws,
                        size_t ws_bytes, void* stream) {
-  msa_status st = check_ws(P, ws, ws_bytes);
+  msa_status st = check_ws(P, ws, ws_bytes, true);
   if (st != MSA_OK) return st;
   if (!s) return MSA_ERR_INVALID_ARG;
   if ((st = check_tensor(Q, s->q_head, s->q_row)) != MSA_OK) return st;
   if ((st = check_tensor(K, s->k_head, s->k_row)) != MSA_OK) return st;
   if ((st = check_tensor(V, s->v_head, s->v_row)) != MSA_OK) return st;
   if (P->ready_ws != ws) return MSA_ERR_STATE;
-  return cuda_status(launch_permute(dev(P, ws), Q, K, V, *s, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_permute(dev(P, ws), Q, K, V, *s, true, static_cast<cudaStream_t>(stream)));
 }
 
 msa_status msa_sparse_prefill(msa_plan* P, const void* Q, const void* K, const void* V, const msa_strides* s,
                               void* ws, size_t ws_bytes, float* lse, void* stream) {
-  msa_status st = check_ws(P, ws, ws_bytes);
+  msa_status st = check_ws(P, ws, ws_bytes, true);
   if (st != MSA_OK) return st;
   if (!s) return MSA_ERR_INVALID_ARG;
   if ((st = check_tensor(Q, s->q_head, s->q_row)) != MSA_OK) return st;
@@ -838,11 +844,29 @@ msa_status msa_sparse_prefill(msa_plan* P, const void* Q, const void* K, const v
   if ((st = check_tensor(V, s->v_head, s->v_row)) != MSA_OK) return st;
   if (lse && reinterpret_cast<uintptr_t>(lse) % 4) return MSA_ERR_ALIGN;
   if (P->ready_ws != ws) return MSA_ERR_STATE;
-  return cuda_status(launch_attention(dev(P, ws), Q, K, V, *s, lse, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_attention(dev(P, ws), Q, K, V, *s, lse, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_sparse_prefill_indexed(msa_plan* P, const void* Q, const void* K, const void* V, void* O,
+                                      const msa_strides* s, void* ws, size_t ws_bytes, float* lse, void* stream) {
+  msa_status st = check_ws(P, ws, ws_bytes, false);
+  if (st != MSA_OK) return st;
+  if (!s) return MSA_ERR_INVALID_ARG;
+  if ((st = check_tensor(Q, s->q_head, s->q_row)) != MSA_OK) return st;
+  if ((st = check_tensor(K, s->k_head, s->k_row)) != MSA_OK) return st;
+  if ((st = check_tensor(V, s->v_head, s->v_row)) != MSA_OK) return st;
+  if ((st = check_tensor(O, s->o_head, s->o_row)) != MSA_OK) return st;
+  if (lse && reinterpret_cast<uintptr_t>(lse) % 4) return MSA_ERR_ALIGN;
+  if (P->ready_ws != ws) return MSA_ERR_STATE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const DevPlan d = dev(P, ws);
+  cudaError_t e = launch_permute(d, Q, K, V, *s, false, cs);  // key gathers only
+  if (e == cudaSuccess) e = launch_attention(d, Q, K, V, *s, lse, O, cs);
+  return cuda_status(e);
 }
 
 msa_status msa_unpermute(msa_plan* P, const void* ws, size_t ws_bytes, void* O, const msa_strides* s, void* stream) {
-  msa_status st = check_ws(P, ws, ws_bytes);
+  msa_status st = check_ws(P, ws, ws_bytes, true);
   if (st != MSA_OK) return st;
   if (!s) return MSA_ERR_INVALID_ARG;
   if ((st = check_tensor(O, s->o_head, s->o_row)) != MSA_OK) return st;

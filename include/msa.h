@@ -126,14 +126,20 @@ typedef struct msa_plan msa_plan;
 msa_status msa_plan_create(const msa_problem* problem, msa_plan** out);
 void msa_plan_destroy(msa_plan* plan);
 
-/* Bytes of device workspace one prefill with this plan needs. */
+/* Bytes of device workspace one prefill with this plan needs (msa_permute, msa_sparse_prefill
+ * and msa_unpermute). */
 size_t msa_workspace_bytes(const msa_plan* plan);
+
+/* Bytes of device workspace the index-based path needs (msa_estimate or msa_set_indices, then
+ * msa_sparse_prefill_indexed): the same layout without its trailing permuted Q and O copies. */
+size_t msa_workspace_bytes_indexed(const msa_plan* plan);
 
 /* Online index estimation (MInference 1.0 "Approach": last-64-query vertical/slash sums,
  * 64-block mean pooling; MMInference "key machinery": grid stride/phase search, per-modality
  * estimation from the 64 latest queries of every modality), followed by the
  * per-head row classes, gathered-key lists, line bitmaps and executed-tile lists.
- * Reads Q and K (device), writes only the workspace. */
+ * Reads Q and K (device), writes only the workspace (ws_bytes >= msa_workspace_bytes_indexed;
+ * the same holds for msa_set_indices). */
 msa_status msa_estimate(msa_plan* plan, const void* Q, const void* K, const msa_strides* strides, void* ws,
                         size_t ws_bytes, void* stream);
 
@@ -173,6 +179,19 @@ msa_status msa_sparse_prefill(msa_plan* plan, const void* Q, const void* K, cons
 /* Scatters the permuted output back to original token order into O (bf16, device). */
 msa_status msa_unpermute(msa_plan* plan, const void* ws, size_t ws_bytes, void* O, const msa_strides* strides,
                          void* stream);
+
+/* Index-based sparse prefill, in place of msa_permute + msa_sparse_prefill + msa_unpermute
+ * (MMInference "core discovery": the permutations are realised as index-based sparse loading
+ * inside the attention kernel).  The query rows of permuted row classes are gathered by row
+ * index from Q into the kernel's query tiles, and every output row is written straight to O
+ * (bf16, device, strides->o_head / o_row) at its original position; the gathered key lines and
+ * the modality-grouped keys are still copied into the workspace first (one pass over K / V).
+ * Same values as the three-call path (same operations in the same order).  lse as for
+ * msa_sparse_prefill.  ws_bytes >= msa_workspace_bytes_indexed; asynchronous on `stream`;
+ * MSA_ERR_STATE if the workspace holds no indices of this plan. */
+msa_status msa_sparse_prefill_indexed(msa_plan* plan, const void* Q, const void* K, const void* V, void* O,
+                                      const msa_strides* strides, void* ws, size_t ws_bytes, float* lse,
+                                      void* stream);
 
 /* ---- inspection (synchronising) ---- */
 

@@ -63,6 +63,18 @@ def test_workspace_grows_with_length():
     assert b > a
 
 
+def test_indexed_workspace_drops_the_permuted_copies():
+    """The index-based path's workspace is the three-call layout without its trailing permuted
+    Q ([n_qslices][LP][128] bf16, at least one slice) and O ([Hq][LP][128] bf16) copies."""
+    import dynamic_sparse_attention_head_b200 as msa
+    import workload
+    for p in (workload.llama3_8b_text(L=4096), workload.qwen2_7b_video_128k()):
+        plan = msa.Plan(p)
+        assert plan.workspace_bytes_indexed < plan.workspace_bytes
+        assert plan.workspace_bytes - plan.workspace_bytes_indexed >= (p.Hq + 1) * p.L * 128 * 2
+        assert plan.workspace_bytes_indexed % 256 == 0
+
+
 def test_attention_units_chunking_rule(monkeypatch):
     """Keys are chunked (65536 per chunk) only when one head's K and V exceed ~96 MB; the
     environment override applies at plan creation."""
