@@ -77,6 +77,7 @@ def _load():
         "msa_tile_stats": ([_P, _P, _P, _P], _I32),
         "msa_attention_units": ([_P, _P], _I32),
         "msa_mask_pairs": ([_P, _P, _P, _P], _I32),
+        "msa_selftest_timeout": ([_P, _P, ctypes.c_uint32, _P], _I32),
         "msa_device_status": ([_P, _P, _P], _I32),
         "msa_status_string": ([_I32], ctypes.c_char_p),
         "msa_kernel_launches": ([], ctypes.c_uint64),
@@ -93,7 +94,7 @@ _lib = _load()
 EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_workspace_bytes_indexed",
            "msa_sparse_prefill_indexed", "msa_estimate", "msa_set_indices",
            "msa_permute", "msa_sparse_prefill", "msa_unpermute", "msa_read_indices", "msa_read_tiles",
-           "msa_tile_stats", "msa_attention_units", "msa_mask_pairs", "msa_device_status", "msa_status_string",
+           "msa_tile_stats", "msa_attention_units", "msa_mask_pairs", "msa_selftest_timeout", "msa_device_status", "msa_status_string",
            "msa_kernel_launches", "msa_vslash_estimate_static")
 
 
@@ -349,6 +350,12 @@ class Plan:
         t = (_I64 * 2)()
         _check("msa_attention_units", _lib.msa_attention_units(self._h, ctypes.cast(t, _P)))
         return int(t[0]), int(t[1])
+
+    def selftest_timeout(self, ws, limit_us: int = 10000, stream=None):
+        """Launch a bounded wait that runs out after limit_us; device_status then reports
+        MSA_ERR_TIMEOUT (7)."""
+        _check("msa_selftest_timeout", _lib.msa_selftest_timeout(self._h, ws.data_ptr(), int(limit_us),
+                                                                 _stream_ptr(stream)))
 
     def device_status(self, ws, stream=None) -> int:
         return int(_lib.msa_device_status(self._h, ws.data_ptr(), _stream_ptr(stream)))

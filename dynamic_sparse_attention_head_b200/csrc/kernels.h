@@ -70,6 +70,8 @@ cudaError_t launch_unpermute(const DevPlan& dp, void* O, const msa_strides& s, c
 // written to O at its original position.
 cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, const void* V, const msa_strides& s,
                              float* lse, void* O, cudaStream_t st);
+// failure-detection self-test: one bounded wait that expires after limit_ns, recorded in *status
+cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 // allowed (query, key) pairs per head over the tile lists, into the workspace's mask_pairs
 cudaError_t launch_mask_count(const DevPlan& dp, cudaStream_t st);
 

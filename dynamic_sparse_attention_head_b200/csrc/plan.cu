@@ -917,6 +917,12 @@ msa_status msa_tile_stats(const msa_plan* P, const void* ws, int64_t tiles[2], v
   return MSA_OK;
 }
 
+msa_status msa_selftest_timeout(const msa_plan* P, void* ws, uint32_t limit_us, void* stream) {
+  if (!P || !ws || limit_us == 0 || limit_us > 1000000u) return MSA_ERR_INVALID_ARG;
+  uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + P->lay.header);
+  return cuda_status(launch_wait_probe(status, (uint64_t)limit_us * 1000ull, static_cast<cudaStream_t>(stream)));
+}
+
 msa_status msa_mask_pairs(const msa_plan* P, void* ws, int64_t* counts, void* stream) {
   if (!P || !ws || !counts) return MSA_ERR_INVALID_ARG;
   if (P->ready_ws != ws) return MSA_ERR_STATE;

@@ -241,8 +241,17 @@ msa_status msa_read_tiles(const msa_plan* plan, const void* ws, int32_t head, in
                           void* stream);
 
 /* Synchronises `stream` and returns the first device-side error recorded in `ws` (MSA_OK if
- * none) and clears it. */
+ * none) and clears it.  The status word is reset by msa_estimate and msa_set_indices (the plan
+ * tables they upload include it); a workspace no call has used yet has no defined status. */
 msa_status msa_device_status(const msa_plan* plan, void* ws, void* stream);
+
+/* Failure-detection self-test.  Every pipeline wait in the library's kernels is bounded by the
+ * global timer; on expiry the kernel records MSA_ERR_TIMEOUT in the workspace's status word and
+ * unwinds (no trap), leaving the context usable.  This call launches one kernel on `stream` whose
+ * bounded wait (the same helper) waits for a barrier no thread arrives at, gives up after
+ * `limit_us` microseconds (1 .. 1000000) and records the timeout the same way; the next
+ * msa_device_status then returns MSA_ERR_TIMEOUT.  Asynchronous. */
+msa_status msa_selftest_timeout(const msa_plan* plan, void* ws, uint32_t limit_us, void* stream);
 
 const char* msa_status_string(msa_status status);
 

@@ -126,3 +126,34 @@ def test_calls_out_of_order_are_refused():
         assert e.value.code == 9  # MSA_ERR_STATE
     plan.estimate(q, k, ws)
     assert plan.mask_pairs(ws).shape == (1,)
+
+
+def test_expired_wait_is_reported_and_the_context_stays_usable():
+    """A bounded wait that nothing completes (msa_selftest_timeout: the kernels' own wait helper
+    on a barrier no thread arrives at) gives up after its limit, is reported as MSA_ERR_TIMEOUT
+    by msa_device_status, is cleared by that call, and leaves the context usable: the rest of the
+    path on the same workspace afterwards still matches the oracle."""
+    import time
+    p = Problem(L=512, Hq=2, Hkv=1, segments=[(0, 512, TEXT)],
+                heads=[Head("vslash", k_v=8, k_s=16), Head("ashape", sink=16, local=64)], name="timeout")
+    Q, K, V = make_inputs(p, seed=21)
+    q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+    plan = msa.Plan(p)
+    ws = plan.alloc_workspace()
+    plan.estimate(q, k, ws)  # uploads the plan tables: the status word starts clear
+    assert plan.device_status(ws) == 0
+    t0 = time.perf_counter()
+    plan.selftest_timeout(ws, limit_us=20000)
+    assert plan.device_status(ws) == 7  # MSA_ERR_TIMEOUT, once the wait ran out
+    elapsed = time.perf_counter() - t0
+    assert 0.015 < elapsed < 5.0, f"wait took {elapsed:.3f} s"
+    assert plan.device_status(ws) == 0  # cleared by the read
+    o = torch.empty_like(q)
+    lse = torch.empty((p.Hq, p.L), dtype=torch.float32, device="cuda")
+    plan.permute(q, k, v, ws)
+    plan.sparse_prefill(q, k, v, ws, lse=lse)
+    plan.unpermute(ws, o)
+    torch.cuda.synchronize()
+    assert plan.device_status(ws) == 0
+    idx = [plan.read_indices(h, ws) for h in range(p.Hq)]
+    _check(p, Q, K, V, idx, o, lse.cpu().numpy(), "after a timeout")
