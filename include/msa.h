@@ -8,7 +8,10 @@
  * from 64-token mean-pooled blocks), Q/K/V are permuted so the selected entries
  * become contiguous, block-sparse causal attention runs over only those blocks,
  * and the output is permuted back.  The four steps are the four calls
- *   msa_estimate -> msa_permute -> msa_sparse_prefill -> msa_unpermute.
+ *   msa_estimate -> msa_permute -> msa_sparse_prefill -> msa_unpermute,
+ * or, with the permutation realised as index-based loading inside the attention
+ * kernel, the two calls
+ *   msa_estimate -> msa_sparse_prefill_indexed.
  *
  * Conventions shared by every call
  *  - Tensors are bf16, d = 128 contiguous elements per row.  Q and O are
@@ -19,13 +22,15 @@
  *  - Causality is always j <= i in ORIGINAL token positions.
  *  - All device pointers are owned by the caller; the library never allocates
  *    or frees device memory.  Scratch lives in one caller-provided workspace of
- *    msa_workspace_bytes() bytes, 256-byte aligned, which carries the estimated
- *    indices and permuted tensors from one call to the next: pass the same
- *    workspace to the four calls of one prefill and do not reuse it for another
- *    prefill until the last call has completed on the stream.
+ *    msa_workspace_bytes() bytes (msa_workspace_bytes_indexed() for the two-call
+ *    path), 256-byte aligned, which carries the estimated indices and permuted
+ *    tensors from one call to the next: pass the same workspace to the calls of
+ *    one prefill and do not reuse it for another prefill until the last call has
+ *    completed on the stream.
  *  - Calls are asynchronous and stream-ordered on the cudaStream_t passed as
- *    `stream` (NULL = legacy default stream); only msa_read_indices,
- *    msa_read_tiles and msa_device_status synchronise.
+ *    `stream` (NULL = legacy default stream); only the inspection calls
+ *    (msa_read_indices, msa_read_tiles, msa_tile_stats, msa_mask_pairs) and
+ *    msa_device_status synchronise.
  *  - Argument errors are returned before any launch.  Conditions found on the
  *    device (a bounded wait that expired, an index outside its buffer) are
  *    recorded in the workspace and reported by msa_device_status; kernels never
@@ -46,7 +51,7 @@ typedef enum {
   MSA_ERR_INVALID_ARG = 1,   /* null pointer, unknown kind, negative budget, ... */
   MSA_ERR_SHAPE = 2,         /* d != 128, L % 64 != 0, Hq % Hkv != 0, segments not tiling [0, L) */
   MSA_ERR_ALIGN = 3,         /* pointer not 16-byte (workspace: 256-byte) aligned, stride not a multiple of 8 */
-  MSA_ERR_WORKSPACE = 4,     /* workspace smaller than msa_workspace_bytes() */
+  MSA_ERR_WORKSPACE = 4,     /* workspace smaller than the call needs (msa_workspace_bytes[_indexed]()) */
   MSA_ERR_UNSUPPORTED = 5,   /* a valid problem outside this build's limits (see msa_status_string) */
   MSA_ERR_CUDA = 6,          /* a CUDA runtime/driver call failed */
   MSA_ERR_TIMEOUT = 7,       /* device: a bounded wait expired (reported by msa_device_status) */
