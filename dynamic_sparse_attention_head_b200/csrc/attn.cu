@@ -90,7 +90,7 @@ struct __align__(1024) AttnSmem {
   uint64_t q_full[N_STREAMS], q_empty[N_STREAMS];
   uint64_t k_full[N_STREAMS], k_empty[N_STREAMS];
   uint64_t v_full[N_STREAMS], v_empty[N_STREAMS];
-  uint64_t qg_full[N_STREAMS];  // Q gathered by the softmax warpgroup (index-based prefill)
+  uint64_t qg_full[N_STREAMS];  // Q gathered by the producer warp (index-based prefill)
   uint64_t s_full[N_STREAMS], p_full[N_STREAMS];
   uint64_t o_full[N_STREAMS], o_free[N_STREAMS];
   // work-item queue of each stream: ids taken from the global counter by the stream's TMA
@@ -438,7 +438,7 @@ __device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, ui
     if (!load_unit(p, e, it, un) || it.ntiles == 0) continue;
     const int n = it.ntiles;
     const bool cont = un.k > 0;  // O starts from the item's accumulator (loaded by the softmax)
-    if (INDEXED && it.q_src) {  // Q gathered by index by the softmax warpgroup
+    if (INDEXED && it.q_src) {  // Q gathered by index by the producer warp
       if (!mbar_wait(&sm.qg_full[s], qg_use & 1, abort)) return;
       ++qg_use;
     } else {
@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
-      mbar_init(&sm.qg_full[s], 128);
+      mbar_init(&sm.qg_full[s], 1);
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 128);
       mbar_init(&sm.o_full[s], 1);
@@ -532,12 +532,26 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // ------------------------------------------------------------------ TMA producers
     // Warp 0 loads stream 0, warp 2 stream 1: two independent load sequences each, polled in
     // turn: Q then the K tiles of every item (slot freed by the QK MMA), and the V tiles
-    // (slot freed by the PV MMA).
-    if (lane == 0) {
+    // (slot freed by the PV MMA).  One lane runs the loop; in the index-based instantiation the
+    // whole warp runs it in step (lane 0 takes every decision that reads shared state and
+    // broadcasts it, and alone issues the copies and arrivals), so that the 32 lanes can gather
+    // the query rows of permuted classes.
+    if (INDEXED || lane == 0) {
+      const bool leader = !INDEXED || lane == 0;
+      // lane 0's value of a condition, for every lane of the warp (index-based instantiation)
+      auto uni = [&](bool x) -> bool {
+        if constexpr (INDEXED) return __shfl_sync(0xFFFFFFFFu, (int)x, 0) != 0;
+        return x;
+      };
+      auto wsync = [&]() {
+        if constexpr (INDEXED) __syncwarp();
+      };
       const int s = warp >> 1;
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      if (leader) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
       const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
       // Work items come from the global counter in plan order (most keys first), one at a
       // time into the stream's queue: the Q/K loads take them as they come, the V loads
@@ -546,15 +560,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       bool ended = false;
       auto publish = [&]() -> bool {
         const uint32_t slot = published % IQ_DEPTH, use = published / IQ_DEPTH;
-        if (ended || (use > 0 && !mbar_test(&sm.iq_empty[s][slot], (use - 1) & 1))) return false;
-        const int id = (int)atomicAdd(p.next_item, 1u);
-        int32_t e[3] = {-1, 0, -1};
-        if (id < p.n_units) unit_entry(p, id, e);
-        ended = e[0] < 0;
-        sm.iq[s][slot][0] = e[0];
-        sm.iq[s][slot][1] = e[1];
-        sm.iq[s][slot][2] = e[2];
-        mbar_arrive(&sm.iq_full[s][slot]);
+        if (ended || uni(use > 0 && !mbar_test(&sm.iq_empty[s][slot], (use - 1) & 1))) return false;
+        int32_t e0 = -1;
+        if (leader) {
+          const int id = (int)atomicAdd(p.next_item, 1u);
+          int32_t e[3] = {-1, 0, -1};
+          if (id < p.n_units) unit_entry(p, id, e);
+          e0 = e[0];
+          sm.iq[s][slot][0] = e[0];
+          sm.iq[s][slot][1] = e[1];
+          sm.iq[s][slot][2] = e[2];
+          mbar_arrive(&sm.iq_full[s][slot]);
+        }
+        if constexpr (INDEXED) {
+          __syncwarp();  // the entry is visible to the whole warp
+          e0 = sm.iq[s][slot][0];
+        }
+        ended = e0 < 0;
         ++published;
         return true;
       };
@@ -562,7 +584,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       int qk_op = -1, v_j = -1;    // -1: no item yet
       ItemInfo qk_it, v_it;
       bool qk_live = true, v_live = true;
-      uint32_t q_iss = 0, k_iss = 0, v_iss = 0;
+      uint32_t q_iss = 0, qt_iss = 0, k_iss = 0, v_iss = 0;  // qt_iss: Q tiles loaded by TMA
       Watchdog wd;
       while (qk_live || v_live) {
         if (qk_live && qk_op < 0) {  // next item of the Q/K loads
@@ -577,27 +599,53 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         if (qk_live && qk_op >= 0) {
           if (qk_op == 0) {
-            if (INDEXED && qk_it.q_src) {  // gathered by the softmax warpgroup; q_empty still
-              ++q_iss;                  // completes once per item
-              qk_op = 1;
-              wd.progress();
-            } else if (q_iss == 0 || mbar_test(&sm.q_empty[s], (q_iss - 1) & 1)) {
-              mbar_arrive_expect_tx(&sm.q_full[s], TILE_BYTES);
-              if (qk_it.q_src) {
-                tma_load_3d(sm.q[s], &tmQp, &sm.q_full[s], 0, qk_it.qrow0 + qk_it.row0, qk_it.q_slice);
-                tma_load_3d(sm.q[s] + ATOM_BYTES, &tmQp, &sm.q_full[s], 64, qk_it.qrow0 + qk_it.row0, qk_it.q_slice);
+            // the slot is free once the stream's previous item's last QK is complete
+            // (q_empty completes once per item)
+            if (uni(q_iss == 0 || mbar_test(&sm.q_empty[s], (q_iss - 1) & 1))) {
+              if (INDEXED && qk_it.q_src) {
+                // the item's query rows from the caller's Q by row index (zeros past the class)
+                // into the 128-byte-swizzled layout the MMA reads: 16-byte chunk c of row r at
+                // chunk c ^ (r & 7); half-warp per row, 64 copies per lane
+                const ClassStatic& cs = class_of(p, qk_it.cls);
+                const int32_t* rows = reinterpret_cast<const int32_t*>(p.ws + cs.rows_off);
+                const uint32_t qs = smem_addr(sm.q[s]);
+                const int ch = lane & 15, a = ch >> 3, c = ch & 7;
+#pragma unroll 2
+                for (int r = lane >> 4; r < TILE; r += 2) {
+                  const int cr = qk_it.row0 + r;
+                  const bool valid = cr < qk_it.nrows;
+                  const int pos = valid ? __ldg(rows + cr) : 0;
+                  const __nv_bfloat16* src = p.qg + (size_t)qk_it.head * p.qg_head + (size_t)pos * p.qg_row + a * 64 + c * 8;
+                  cp_async16_zfill(qs + a * ATOM_BYTES + (uint32_t)r * 128u + ((uint32_t)(c ^ (r & 7)) << 4), src,
+                                   valid ? 16u : 0u);
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                wsync();
+                if (leader) mbar_arrive(&sm.qg_full[s]);
               } else {
-                tma_load_3d(sm.q[s], &tmQ, &sm.q_full[s], 0, qk_it.row0, qk_it.head);
-                tma_load_3d(sm.q[s] + ATOM_BYTES, &tmQ, &sm.q_full[s], 64, qk_it.row0, qk_it.head);
+                if (leader) {
+                  mbar_arrive_expect_tx(&sm.q_full[s], TILE_BYTES);
+                  if (qk_it.q_src) {
+                    tma_load_3d(sm.q[s], &tmQp, &sm.q_full[s], 0, qk_it.qrow0 + qk_it.row0, qk_it.q_slice);
+                    tma_load_3d(sm.q[s] + ATOM_BYTES, &tmQp, &sm.q_full[s], 64, qk_it.qrow0 + qk_it.row0,
+                                qk_it.q_slice);
+                  } else {
+                    tma_load_3d(sm.q[s], &tmQ, &sm.q_full[s], 0, qk_it.row0, qk_it.head);
+                    tma_load_3d(sm.q[s] + ATOM_BYTES, &tmQ, &sm.q_full[s], 64, qk_it.row0, qk_it.head);
+                  }
+                }
+                ++qt_iss;
               }
               ++q_iss;
               qk_op = 1;
               wd.progress();
             }
-          } else if (k_iss == 0 || mbar_test(&sm.k_empty[s], (k_iss - 1) & 1)) {
+          } else if (uni(k_iss == 0 || mbar_test(&sm.k_empty[s], (k_iss - 1) & 1))) {
             const int j = qk_op - 1;
-            issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, false, __ldg(tiles + qk_it.tile0 + j), qk_it, sm.k[s],
-                     &sm.k_full[s]);
+            if (leader)
+              issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, false, __ldg(tiles + qk_it.tile0 + j), qk_it, sm.k[s],
+                       &sm.k_full[s]);
             ++k_iss;
             wd.progress();
             if (j + 1 == qk_it.ntiles) {
@@ -613,31 +661,35 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           const int32_t* e = sm.iq[s][slot];
           UnitInfo un;
           if (e[0] < 0) {
-            mbar_arrive(&sm.iq_empty[s][slot]);
+            if (leader) mbar_arrive(&sm.iq_empty[s][slot]);
             v_live = false;
           } else if (!load_unit(p, e, v_it, un) || v_it.ntiles == 0) {
-            mbar_arrive(&sm.iq_empty[s][slot]);
+            if (leader) mbar_arrive(&sm.iq_empty[s][slot]);
             ++v_q;
           } else {
             v_j = 0;
           }
         }
-        if (v_live && v_j >= 0 && (v_iss == 0 || mbar_test(&sm.v_empty[s], (v_iss - 1) & 1))) {
-          issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, true, __ldg(tiles + v_it.tile0 + v_j), v_it, sm.v[s],
-                   &sm.v_full[s]);
+        if (v_live && v_j >= 0 && uni(v_iss == 0 || mbar_test(&sm.v_empty[s], (v_iss - 1) & 1))) {
+          if (leader)
+            issue_kv(&tmK, &tmV, &tmK2, &tmV2, &tmXK, &tmXV, true, __ldg(tiles + v_it.tile0 + v_j), v_it, sm.v[s],
+                     &sm.v_full[s]);
           ++v_iss;
           wd.progress();
           if (++v_j == v_it.ntiles) {
-            mbar_arrive(&sm.iq_empty[s][v_q % IQ_DEPTH]);
+            if (leader) mbar_arrive(&sm.iq_empty[s][v_q % IQ_DEPTH]);
             ++v_q;
             v_j = -1;
           }
         }
-        if (wd.expired(abort)) {
+        if (uni(wd.expired(abort))) {
           // let the copies already issued land before the CTA goes away
-          if (q_iss) mbar_wait(&sm.q_full[s], (q_iss - 1) & 1, abort, 100000000ull);
-          if (k_iss) mbar_wait(&sm.k_full[s], (k_iss - 1) & 1, abort, 100000000ull);
-          if (v_iss) mbar_wait(&sm.v_full[s], (v_iss - 1) & 1, abort, 100000000ull);
+          if (leader) {
+            if (qt_iss) mbar_wait(&sm.q_full[s], (qt_iss - 1) & 1, abort, 100000000ull);
+            if (k_iss) mbar_wait(&sm.k_full[s], (k_iss - 1) & 1, abort, 100000000ull);
+            if (v_iss) mbar_wait(&sm.v_full[s], (v_iss - 1) & 1, abort, 100000000ull);
+          }
+          wsync();
           break;
         }
       }
@@ -696,23 +748,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         continue;
       }
 
-      if (INDEXED && it.q_src) {
-        // Q row t of the unit from the caller's Q at its original position (zeros for rows past
-        // the class) into the stream's Q slot in the 128-byte-swizzled layout the MMA reads:
-        // 16-byte chunk c of row t at chunk c ^ (t & 7).  The slot is free: this warpgroup has
-        // read the S of the stream's previous unit, so its last QK is complete.
-        const __nv_bfloat16* src = p.qg + (size_t)it.head * p.qg_head + (size_t)rc.qpos * p.qg_row;
-        const uint32_t bytes = rc.valid ? 16u : 0u;
-        const uint32_t dst = smem_addr(sm.q[s]) + (uint32_t)t * 128u;
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            cp_async16_zfill(dst + a * ATOM_BYTES + ((uint32_t)(c ^ (t & 7)) << 4), src + a * 64 + c * 8, bytes);
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(&sm.qg_full[s]);
-      }
       float m_used = -INFINITY, l = 0.f;
       // A unit after the item's first key chunk resumes from the item's accumulator: the
       // previous chunk's unit releases it (chunk_done) once every row is stored.
