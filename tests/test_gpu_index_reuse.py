@@ -1,4 +1,5 @@
-"""Index reuse across layers of one layout: the index sets and tile lists
+"""Index reuse across layers of one layout (MMInference: an index estimated once per modality
+layout serves the later layers and segments of that layout): the index sets and tile lists
 a msa_estimate leaves in the workspace serve a later layer with other Q/K/V of the same layout
 (permute -> sparse prefill -> unpermute without estimating again); that layer's output must be
 the oracle's masked attention under the first layer's index sets."""
