@@ -1,0 +1,91 @@
+"""Seeded random small layers through the whole path against the oracle: segment layouts (one
+to six runs of text and video of random lengths), GQA group sizes, head kinds and budgets drawn
+at random.  Per layer: the device's index sets against the oracle's (near-tie rule), the output
+and lse against the oracle's masked attention under the device's index sets, the device's count
+of allowed pairs against the oracle's masks (exact), and the index-based path bit-identical to
+the three-call path."""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import compare_outputs, to_dev
+from test_gpu_estimate import _check_head
+from workload import TEXT, VIDEO, Head, Problem, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import dynamic_sparse_attention_head_b200 as msa  # noqa: E402
+
+N_CASES = 48
+
+
+def random_problem(seed: int) -> Problem:
+    rng = np.random.default_rng(1000 + seed)
+    L = 64 * int(rng.integers(1, 33))  # 64 .. 2048
+    nseg = int(rng.integers(1, 7))
+    cuts = np.sort(rng.choice(np.arange(1, L), size=nseg - 1, replace=False)) if nseg > 1 else np.array([], int)
+    bounds = [0] + [int(c) for c in cuts] + [L]
+    segs = [(bounds[i], bounds[i + 1] - bounds[i], int(rng.integers(0, 2))) for i in range(nseg)]
+    has_video = any(m == VIDEO for _, _, m in segs)
+    fs = int(rng.choice([16, 24, 32, 48, 64]))
+    Hkv = int(rng.integers(1, 3))
+    Hq = Hkv * int(rng.integers(1, 4))
+    kinds = ["dense", "ashape", "vslash", "block", "qbound", "bound2d"] + (["grid"] if has_video else [])
+    heads = []
+    for _ in range(Hq):
+        k = str(rng.choice(kinds))
+        if k == "ashape":
+            heads.append(Head(k, sink=int(rng.integers(0, 129)), local=int(rng.integers(1, 513))))
+        elif k in ("vslash", "qbound", "bound2d"):
+            heads.append(Head(k, k_v=int(rng.integers(1, L // 4 + 1)), k_s=int(rng.integers(1, L // 2 + 1))))
+        elif k == "block":
+            if rng.random() < 0.5:
+                heads.append(Head(k, topk_blocks=int(rng.integers(1, 7))))
+            else:
+                heads.append(Head(k, block_budget=float(rng.uniform(0.05, 0.6))))
+        elif k == "grid":
+            if rng.random() < 0.5:
+                heads.append(Head(k, strides=(fs,), n_phases=int(rng.integers(1, 4))))
+            else:
+                heads.append(Head(k, strides=(fs,), grid_budget=float(rng.uniform(0.05, 0.3))))
+        else:
+            heads.append(Head(k))
+    return Problem(L=L, Hq=Hq, Hkv=Hkv, segments=segs, heads=heads, frame_stride=fs, name=f"random{seed}")
+
+
+@pytest.mark.parametrize("seed", range(N_CASES))
+def test_random_layer(seed):
+    p = random_problem(seed)
+    what = f"{p.name} (L={p.L}, Hq={p.Hq}, Hkv={p.Hkv}, segments={p.segments}, kinds={[h.kind for h in p.heads]})"
+    Q, K, V = make_inputs(p, seed=seed)
+    q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+    plan = msa.Plan(p)
+    ws = plan.alloc_workspace()
+    o = torch.empty_like(q)
+    lse = torch.empty((p.Hq, p.L), dtype=torch.float32, device="cuda")
+    plan.forward(q, k, v, ws, o, lse=lse)
+    torch.cuda.synchronize()
+    assert plan.device_status(ws) == 0, what
+    idx = [plan.read_indices(h, ws) for h in range(p.Hq)]
+    for h in range(p.Hq):
+        _check_head(p, h, idx[h], oracle.estimate_head(p, h, Q, K))
+    Oref, lref = oracle.attention(p, Q, K, V, idx)
+    got, lse_h = o.float().cpu().numpy(), lse.cpu().numpy()
+    for h in range(p.Hq):
+        compare_outputs(got[h], Oref[h], f"{what} head {h}")
+        fin = np.isfinite(lref[h])
+        assert np.array_equal(fin, np.isfinite(lse_h[h])), f"{what} head {h}: empty rows differ"
+        np.testing.assert_allclose(lse_h[h][fin], lref[h][fin], atol=2e-3, rtol=1e-3)
+    pairs = [int(oracle.mask_count(p, h, idx[h]).sum()) for h in range(p.Hq)]
+    assert plan.mask_pairs(ws).tolist() == pairs, what
+    ws_i = plan.alloc_workspace(indexed=True)
+    o_i = torch.empty_like(q)
+    lse_i = torch.empty_like(lse)
+    plan.forward(q, k, v, ws_i, o_i, lse=lse_i, indexed=True)
+    torch.cuda.synchronize()
+    assert plan.device_status(ws_i) == 0, what
+    assert torch.equal(o, o_i) and torch.equal(lse, lse_i), f"{what}: index-based path differs"
