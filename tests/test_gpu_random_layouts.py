@@ -3,7 +3,8 @@ to six runs of text and video of random lengths), GQA group sizes, head kinds an
 at random.  Per layer: the device's index sets against the oracle's (near-tie rule), the output
 and lse against the oracle's masked attention under the device's index sets, the device's count
 of allowed pairs against the oracle's masks (exact), and the index-based path bit-identical to
-the three-call path."""
+the three-call path.  Every third layer runs with its keys cut into small chunks (the
+long-sequence path)."""
 import numpy as np
 import pytest
 
@@ -58,12 +59,19 @@ def random_problem(seed: int) -> Problem:
 
 
 @pytest.mark.parametrize("seed", range(N_CASES))
-def test_random_layer(seed):
+def test_random_layer(seed, monkeypatch):
     p = random_problem(seed)
-    what = f"{p.name} (L={p.L}, Hq={p.Hq}, Hkv={p.Hkv}, segments={p.segments}, kinds={[h.kind for h in p.heads]})"
+    chunk = 0
+    if seed % 3 == 0 and p.L > 128:  # keys cut into small chunks (the long-sequence path)
+        chunk = 128 * int(np.random.default_rng(seed).integers(1, (p.L - 1) // 128 + 1))
+        monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", str(chunk))
+    what = (f"{p.name} (L={p.L}, Hq={p.Hq}, Hkv={p.Hkv}, segments={p.segments}, "
+            f"kinds={[h.kind for h in p.heads]}, key chunk={chunk or 'none'})")
     Q, K, V = make_inputs(p, seed=seed)
     q, k, v = to_dev(Q), to_dev(K), to_dev(V)
     plan = msa.Plan(p)
+    if chunk:
+        assert plan.attention_units()[1] == (p.L + chunk - 1) // chunk > 1, what
     ws = plan.alloc_workspace()
     o = torch.empty_like(q)
     lse = torch.empty((p.Hq, p.L), dtype=torch.float32, device="cuda")
