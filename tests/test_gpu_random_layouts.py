@@ -97,3 +97,59 @@ def test_random_layer(seed, monkeypatch):
     torch.cuda.synchronize()
     assert plan.device_status(ws_i) == 0, what
     assert torch.equal(o, o_i) and torch.equal(lse, lse_i), f"{what}: index-based path differs"
+
+
+def random_medium_problem(seed: int) -> Problem:
+    """8K-32K tokens, up to 12 text / video runs, frame strides up to 256."""
+    rng = np.random.default_rng(5000 + seed)
+    L = 1024 * int(rng.integers(8, 33))
+    nseg = int(rng.integers(1, 13))
+    cuts = np.sort(rng.choice(np.arange(1, L), size=nseg - 1, replace=False)) if nseg > 1 else np.array([], int)
+    bounds = [0] + [int(c) for c in cuts] + [L]
+    segs = [(bounds[i], bounds[i + 1] - bounds[i], VIDEO if i % 2 == (seed & 1) else TEXT) for i in range(nseg)]
+    has_video = any(m == VIDEO for _, _, m in segs)
+    fs = int(rng.choice([64, 128, 196, 256]))
+    Hkv = int(rng.integers(1, 3))
+    Hq = Hkv * int(rng.integers(1, 4))
+    kinds = ["ashape", "vslash", "block", "qbound", "bound2d"] + (["grid"] if has_video else [])
+    heads = []
+    for _ in range(Hq):
+        k = str(rng.choice(kinds))
+        if k == "ashape":
+            heads.append(Head(k, sink=128, local=int(64 * rng.integers(1, 33))))
+        elif k in ("vslash", "qbound", "bound2d"):
+            heads.append(Head(k, k_v=int(rng.integers(50, 1001)), k_s=int(rng.integers(100, 3001))))
+        elif k == "block":
+            heads.append(Head(k, block_budget=float(rng.uniform(0.02, 0.2))))
+        else:
+            heads.append(Head(k, strides=(fs,), grid_budget=float(rng.uniform(0.02, 0.15))))
+    return Problem(L=L, Hq=Hq, Hkv=Hkv, segments=segs, heads=heads, frame_stride=fs, name=f"medium{seed}")
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_medium_layer(seed):
+    """Medium random layers: index sets against the oracle, outputs on sampled rows (every
+    segment's first and last rows, the sequence's last 64, seeded random rows)."""
+    p = random_medium_problem(seed)
+    what = f"{p.name} (L={p.L}, Hq={p.Hq}, Hkv={p.Hkv}, {len(p.segments)} segments, kinds={[h.kind for h in p.heads]})"
+    Q, K, V = make_inputs(p, seed=seed)
+    q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+    plan = msa.Plan(p)
+    ws = plan.alloc_workspace()
+    o = torch.empty_like(q)
+    plan.forward(q, k, v, ws, o)
+    torch.cuda.synchronize()
+    assert plan.device_status(ws) == 0, what
+    idx = [plan.read_indices(h, ws) for h in range(p.Hq)]
+    for h in range(p.Hq):
+        _check_head(p, h, idx[h], oracle.estimate_head(p, h, Q, K))
+    rng = np.random.default_rng(seed)
+    rows = {p.L - 1 - i for i in range(64)}
+    for (s0, n, _m) in p.segments:
+        rows.update([s0, s0 + n - 1])
+    rows.update(rng.choice(p.L, size=96, replace=False).tolist())
+    rows = np.array(sorted(rows))
+    got = o[:, torch.as_tensor(rows, device=o.device)].float().cpu().numpy()
+    for h in range(p.Hq):
+        ref, _ = oracle.attention_head(p, h, Q, K, V, idx[h], rows)
+        compare_outputs(got[h], ref, f"{what} head {h}")
