@@ -157,3 +157,36 @@ def test_expired_wait_is_reported_and_the_context_stays_usable():
     assert plan.device_status(ws) == 0
     idx = [plan.read_indices(h, ws) for h in range(p.Hq)]
     _check(p, Q, K, V, idx, o, lse.cpu().numpy(), "after a timeout")
+
+
+def test_concurrent_prefills_on_two_streams():
+    """All device state lives in the caller's workspace (work counters, index sets, tile lists,
+    status word), so two layers on two streams, each with its own workspace, may run at the same
+    time: each output equals its sequential run bit for bit."""
+    P = [Problem(L=1472, Hq=7, Hkv=1, segments=[(0, 576, VIDEO), (576, 256, TEXT), (832, 480, VIDEO), (1312, 160, TEXT)],
+                 heads=ALL_KINDS, frame_stride=32, name="streams-a"),
+         Problem(L=2048, Hq=4, Hkv=2, segments=[(0, 2048, TEXT)],
+                 heads=[Head("vslash", k_v=40, k_s=200), Head("ashape", sink=64, local=256),
+                        Head("block", topk_blocks=4), Head("dense")], name="streams-b")]
+    runs = []
+    for p in P:
+        Q, K, V = make_inputs(p, seed=31)
+        plan = msa.Plan(p)
+        runs.append((p, plan, plan.alloc_workspace(), to_dev(Q), to_dev(K), to_dev(V)))
+    seq = []
+    for p, plan, ws, q, k, v in runs:
+        o = torch.empty_like(q)
+        plan.forward(q, k, v, ws, o)
+        torch.cuda.synchronize()
+        assert plan.device_status(ws) == 0
+        seq.append(o)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.empty_like(r[3]) for r in runs]
+    for _ in range(3):
+        for (p, plan, ws, q, k, v), o, st in zip(runs, outs, streams):
+            with torch.cuda.stream(st):
+                plan.forward(q, k, v, ws, o, stream=st)
+        torch.cuda.synchronize()
+        for (p, plan, ws, *_), o, ref in zip(runs, outs, seq):
+            assert plan.device_status(ws) == 0
+            assert torch.equal(o, ref), f"{p.name}: concurrent run differs"
