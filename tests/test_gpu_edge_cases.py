@@ -190,3 +190,42 @@ def test_concurrent_prefills_on_two_streams():
         for (p, plan, ws, *_), o, ref in zip(runs, outs, seq):
             assert plan.device_status(ws) == 0
             assert torch.equal(o, ref), f"{p.name}: concurrent run differs"
+
+
+def test_path_replays_from_a_cuda_graph():
+    """The whole per-layer path (estimate -> permute -> sparse prefill -> unpermute, and the
+    index-based pair) is stream-ordered with no synchronisation, so it can be captured in a CUDA
+    graph; replays with new inputs copied into the captured buffers match eager runs bit for bit."""
+    p = Problem(L=1472, Hq=7, Hkv=1, segments=[(0, 576, VIDEO), (576, 256, TEXT), (832, 480, VIDEO), (1312, 160, TEXT)],
+                heads=ALL_KINDS, frame_stride=32, name="graph")
+    plan = msa.Plan(p)
+    for indexed in (False, True):
+        ws = plan.alloc_workspace(indexed=indexed)
+        inputs = [make_inputs(p, seed=s) for s in (41, 42)]
+        q, k, v = (to_dev(x) for x in inputs[0])
+        o = torch.empty_like(q)
+        eager = []
+        for Q, K, V in inputs:
+            qq, kk, vv = to_dev(Q), to_dev(K), to_dev(V)
+            oo = torch.empty_like(qq)
+            plan.forward(qq, kk, vv, ws, oo, indexed=indexed)
+            torch.cuda.synchronize()
+            eager.append(oo)
+        st = torch.cuda.Stream()
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):  # warm-up on the capture stream
+            plan.forward(q, k, v, ws, o, stream=st, indexed=indexed)
+        torch.cuda.current_stream().wait_stream(st)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            plan.forward(q, k, v, ws, o, stream=st, indexed=indexed)
+        for (Q, K, V), ref in zip(inputs, eager):
+            q.copy_(to_dev(Q))
+            k.copy_(to_dev(K))
+            v.copy_(to_dev(V))
+            g.replay()
+            torch.cuda.synchronize()
+            assert plan.device_status(ws) == 0
+            assert torch.equal(o, ref), f"graph replay differs (indexed={indexed})"
+        del g
