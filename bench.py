@@ -17,6 +17,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -178,11 +179,21 @@ def make_host_inputs(p, seed):
     return Q, K, V
 
 
+_COMMENT_OR_STRING = re.compile(r'("(?:\\.|[^"\\])*")|//[^\n]*|/\*.*?\*/', re.S)
+
+
+def code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and with whitespace runs collapsed."""
+    return " ".join(_COMMENT_OR_STRING.sub(lambda m: m.group(1) or " ", text).split())
+
+
 def attn_source_hash():
+    """Identity of the attention kernel's code (comments and layout excluded): the recorded DRAM
+    traffic is valid only for the code it was measured on."""
     h = hashlib.sha256()
     for f in ("attn.cu", "ptx.cuh", "msa_internal.h", "plan.cu"):  # plan.cu: work-item order
-        with open(os.path.join(ROOT, "dynamic_sparse_attention_head_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "dynamic_sparse_attention_head_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

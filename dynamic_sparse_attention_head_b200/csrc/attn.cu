@@ -11,7 +11,9 @@
 //    accumulator in the workspace (unnormalised O, running max and sum), handed over between
 //    units through a per-item counter (release / acquire);
 //  - warps 0 and 2 stream the Q, K and V tiles of stream 0 and 1 with TMA (128-byte
-//    swizzle) into single-buffered slots of their own;
+//    swizzle) into single-buffered slots of their own; in the index-based instantiation
+//    (msa_attn_kernel<true>) the whole warp also gathers the query rows of permuted classes
+//    from the caller's Q by row index (cp.async into the swizzled Q slot);
 //  - warps 1 and 3 (one thread each) issue the tcgen05.mma of stream 0 and 1:
 //    S_s = Q_s K^T into stream s's TMEM columns, then O_s += P_s V with P_s read from TMEM
 //    and O_s resident in TMEM for the whole unit; a group [PV(j), QK(j + 1)] is issued under
@@ -22,7 +24,8 @@
 //    thread and all 128 keys of every tile: they read S with tcgen05.ld, apply the element
 //    mask (causal in original positions + the head's pattern), run the online softmax in fp32
 //    (exp2 on MUFU, lazy rescale of O when the running max grows by more than 2^8), write P
-//    as packed bf16 over the first 64 columns of S with tcgen05.st, and finally normalise O.
+//    as packed bf16 over the first 64 columns of S with tcgen05.st, and finally normalise O
+//    into the permuted O copy (or, index-based, into the caller's O at the original position).
 // Every wait is bounded; on a timeout the CTA records DEV_ERR_TIMEOUT and unwinds.
 #include <cuda.h>
 #include <cuda_bf16.h>
