@@ -45,3 +45,20 @@ def test_job_totals_single_rank_is_identity():
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     import bench
     assert bench.job_totals(7.5, 42.0, 1) == (7.5, 42.0)
+
+
+def test_kernel_code_hash_ignores_comments_only():
+    """The identity under which the recorded DRAM traffic stays valid: comments and layout do not
+    change it, code (including inline-PTX strings) does."""
+    import importlib.util
+    import os
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(os.path.dirname(__file__), "..", "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    src = 'int f(int x) {  // doubles\n  /* a\n block */ return 2 * x;\n}\nasm("add.s32 %0, %1; // not a comment");\n'
+    same = 'int f(int x)\n{ return 2 * x; }   // other words\nasm("add.s32 %0, %1; // not a comment");'
+    other = 'int f(int x) { return 3 * x; }\nasm("add.s32 %0, %1; // not a comment");'
+    ptx = 'int f(int x) { return 2 * x; }\nasm("sub.s32 %0, %1; // not a comment");'
+    assert b.code_only(src) == b.code_only(same)
+    assert b.code_only(src) != b.code_only(other)
+    assert b.code_only(src) != b.code_only(ptx)
