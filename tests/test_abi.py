@@ -90,3 +90,40 @@ def test_attention_units_chunking_rule(monkeypatch):
     monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", "0")
     units, chunks = msa.Plan(p).attention_units()
     assert chunks == 1
+
+
+def test_workspace_size_and_state_checks_come_before_any_device_access():
+    """The size, alignment and call-order checks of the calls return before anything touches
+    device memory, so they are exercised here with placeholder addresses (never dereferenced)."""
+    import ctypes
+    import dynamic_sparse_attention_head_b200 as msa
+    from dynamic_sparse_attention_head_b200 import _lib, Strides
+    from workload import llama3_8b_text
+
+    plan = msa.Plan(llama3_8b_text(L=4096))
+    full, indexed = plan.workspace_bytes, plan.workspace_bytes_indexed
+    assert indexed < full
+    ws, q, k, v, o = 1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20  # aligned placeholders
+    s = Strides()
+    for name in ("q", "k", "v", "o"):
+        setattr(s, f"{name}_head", 4096 * 128)
+        setattr(s, f"{name}_row", 128)
+    sp = ctypes.byref(s)
+    WORKSPACE, ALIGN, STATE = 4, 3, 9
+    # the index-based path needs only its own size; the three-call path the full one
+    assert _lib.msa_estimate(plan._h, q, k, sp, ws, indexed - 256, None) == WORKSPACE
+    assert _lib.msa_sparse_prefill_indexed(plan._h, q, k, v, o, sp, ws, indexed - 256, None, None) == WORKSPACE
+    assert _lib.msa_permute(plan._h, q, k, v, sp, ws, indexed, None) == WORKSPACE
+    assert _lib.msa_sparse_prefill(plan._h, q, k, v, sp, ws, indexed, None, None) == WORKSPACE
+    assert _lib.msa_unpermute(plan._h, ws, indexed, o, sp, None) == WORKSPACE
+    # alignment
+    assert _lib.msa_sparse_prefill_indexed(plan._h, q, k, v, o, sp, ws + 128, indexed, None, None) == ALIGN
+    assert _lib.msa_sparse_prefill_indexed(plan._h, q, k, v, o + 8, sp, ws, indexed, None, None) == ALIGN
+    # no indices in this workspace yet: the prefill and the pair count refuse it
+    assert _lib.msa_sparse_prefill_indexed(plan._h, q, k, v, o, sp, ws, indexed, None, None) == STATE
+    counts = (ctypes.c_int64 * plan.problem.Hq)()
+    assert _lib.msa_mask_pairs(plan._h, ws, None, None) == 1  # no output buffer
+    assert _lib.msa_mask_pairs(plan._h, ws, ctypes.cast(counts, ctypes.c_void_p), None) == STATE
+    # the self-test's limit is bounded to (0, 1 s]
+    assert _lib.msa_selftest_timeout(plan._h, ws, 0, None) == 1
+    assert _lib.msa_selftest_timeout(plan._h, ws, 2000000, None) == 1
