@@ -67,6 +67,8 @@ def _load():
         lib.orc_mask_count.argtypes = [ctypes.POINTER(_Mask), _P, _I64, _P]
         lib.orc_attention.argtypes = [_P, _P, _P, _I64, ctypes.c_int, ctypes.c_float, ctypes.POINTER(_Mask),
                                       _P, _I64, _P, _P]
+        lib.orc_attention_permuted.argtypes = [_P, _P, _P, _P, _I64, _P, _I64, ctypes.c_int, ctypes.c_float,
+                                               ctypes.POINTER(_Mask), _P, _P]
         _lib = lib
     return _lib
 
@@ -380,3 +382,67 @@ def attention_head(p: Problem, h: int, Q, K, V, idx: Dict, rows=None):
 def attention(p: Problem, Q, K, V, idx: List[Dict], rows=None):
     outs = [attention_head(p, h, Q, K, V, idx[h], rows) for h in range(p.Hq)]
     return np.stack([o for o, _ in outs]), np.stack([l for _, l in outs])
+
+
+# --------------------------------------------------------------------------------------
+# permutation (MMInference review page, "key machinery" and "core discovery")
+# --------------------------------------------------------------------------------------
+def _front(first: np.ndarray) -> np.ndarray:
+    """Stable partition of positions 0..L-1: those with first[t] true, then the rest, each
+    in ascending order."""
+    first = np.asarray(first, bool)
+    return np.concatenate([np.nonzero(first)[0], np.nonzero(~first)[0]]).astype(np.int64)
+
+
+def permutation(p: Problem, h: int, idx: Dict):
+    """The row and column permutation of q-head h, as arrays of original positions in permuted
+    order (qperm[r] = original query position of permuted row r; likewise kperm for keys).
+
+    Readings (the pages state the goal, contiguous selected entries, not an ordering):
+      grid (Algorithm 1): queries and keys on the selected grid lines first, then the others;
+      Q-boundary (Algorithm 2): queries grouped by modality (text, then video), keys unchanged;
+      2D-boundary (Algorithm 3): queries and keys grouped by modality;
+      vertical-slash: keys on the vertical lines first (the lines gathered), queries unchanged;
+      other kinds: identity.
+    Every group keeps ascending original order."""
+    kind = p.heads[h].kind
+    L = p.L
+    ident = np.arange(L, dtype=np.int64)
+    mod = p.modality()
+    if kind == "grid":
+        g = grid_marks(p, idx["stride"], idx["phases"]).astype(bool)
+        return _front(g), _front(g)
+    if kind == "qbound":
+        return _front(mod == TEXT), ident
+    if kind == "bound2d":
+        return _front(mod == TEXT), _front(mod == TEXT)
+    if kind == "vslash":
+        v = np.zeros(L, bool)
+        v[np.asarray(idx["V"], np.int64)] = True
+        return ident, _front(v)
+    return ident, ident
+
+
+def attention_permuted(p: Problem, h: int, Q, K, V, idx: Dict, qperm, kperm):
+    """Permute -> attend -> unpermute for q-head h: gather Q rows by qperm and K/V rows by
+    kperm, run the masked attention in permuted coordinates with the mask evaluated through
+    the original positions, and scatter the output rows back to their original positions.
+    Returns (O [L, d] fp32, lse [L] fp32) in original order."""
+    lib = _load()
+    kvh = h // (p.Hq // p.Hkv)
+    qperm = _c(qperm, np.int64)
+    kperm = _c(kperm, np.int64)
+    Qp = _c(np.asarray(Q[h])[qperm], np.uint16)
+    Kp = _c(np.asarray(K[kvh])[kperm], np.uint16)
+    Vp = _c(np.asarray(V[kvh])[kperm], np.uint16)
+    Op = np.zeros((len(qperm), p.d), np.float32)
+    lp = np.zeros(len(qperm), np.float32)
+    ma = MaskArrays(p, h, idx)
+    lib.orc_attention_permuted(Qp.ctypes.data, Kp.ctypes.data, Vp.ctypes.data, qperm.ctypes.data, len(qperm),
+                               kperm.ctypes.data, len(kperm), p.d, p.scale, ctypes.byref(ma.mask),
+                               Op.ctypes.data, lp.ctypes.data)
+    O = np.zeros((p.L, p.d), np.float32)
+    lse = np.full(p.L, -np.inf, np.float32)
+    O[qperm] = Op
+    lse[qperm] = lp
+    return O, lse

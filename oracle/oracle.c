@@ -295,3 +295,59 @@ void orc_attention(const uint16_t* Qh, const uint16_t* Kh, const uint16_t* Vh, i
     free(acc);
   }
 }
+
+/*
+ * Masked attention taken in permuted coordinates (MMInference review page, "core
+ * discovery": the permutation is realised as index-based loading, so the output of a
+ * head does not change; "key machinery": grid, Q-boundary and 2D-boundary heads
+ * permute the query and key axes so that the selected entries become contiguous).
+ *
+ * Row r of Qp is the query at original position qpos[r]; row t of Kp and Vp is the key
+ * at original position kpos[t].  Causality and the head's pattern are evaluated
+ * through the original positions, allowed(qpos[r], kpos[t]); the keys are visited in
+ * permuted order t = 0 .. nk - 1.  Output row r (and lse[r]) belongs to original
+ * position qpos[r]: the caller scatters it back.  Same arithmetic as orc_attention
+ * except for the order of the fp64 sums.
+ */
+void orc_attention_permuted(const uint16_t* Qp, const uint16_t* Kp, const uint16_t* Vp,
+                            const int64_t* qpos, int64_t nq, const int64_t* kpos, int64_t nk, int d,
+                            float scale, const orc_mask* m, float* Op, float* lse) {
+#pragma omp parallel
+  {
+    float* x = (float*)malloc(sizeof(float) * (size_t)(nk > 0 ? nk : 1));
+    int64_t* ts = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nk > 0 ? nk : 1));
+    double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 8)
+    for (int64_t r = 0; r < nq; ++r) {
+      const int64_t i = qpos[r];
+      const uint16_t* q = Qp + (size_t)r * d;
+      int64_t n = 0;
+      float mx = -INFINITY;
+      for (int64_t t = 0; t < nk; ++t) {
+        if (!allowed(m, i, kpos[t])) continue;
+        ts[n] = t;
+        x[n] = logit(q, Kp + (size_t)t * d, d, scale);
+        if (x[n] > mx) mx = x[n];
+        ++n;
+      }
+      if (n == 0) {
+        for (int c = 0; c < d; ++c) Op[r * d + c] = 0.0f;
+        lse[r] = -INFINITY;
+        continue;
+      }
+      for (int c = 0; c < d; ++c) acc[c] = 0.0;
+      double Z = 0.0;
+      for (int64_t u = 0; u < n; ++u) {
+        double p = exp((double)x[u] - (double)mx);
+        Z += p;
+        const uint16_t* vr = Vp + (size_t)ts[u] * d;
+        for (int c = 0; c < d; ++c) acc[c] += p * bf(vr[c]);
+      }
+      for (int c = 0; c < d; ++c) Op[r * d + c] = (float)(acc[c] / Z);
+      lse[r] = (float)((double)mx + log(Z));
+    }
+    free(x);
+    free(ts);
+    free(acc);
+  }
+}

@@ -72,9 +72,16 @@ def compare_outputs(got: np.ndarray, ref: np.ndarray, what: str = ""):
     return mae, rel
 
 
-def near_tie_ok(got, ref, scores, cand=None, what=""):
-    """Index sets must be identical except for swaps among candidates whose (fp32) oracle
-    scores lie within TIE_REL of the k-th score, relative to the largest candidate score."""
+def near_tie_ok(got, ref, scores, cand=None, what="", relative_to="tau"):
+    """Index sets must be identical except for swaps among near-tied candidates: every index in
+    the symmetric difference must have an (fp32) oracle score within TIE_REL of the k-th
+    selected score tau.
+
+    relative_to="tau" (probability sums: vertical, slash, grid phase means, all positive):
+    the bound is TIE_REL * |tau|, floored at TIE_REL * 1e-3 * max|candidate score| so that a
+    k-th score that is itself a rounding-level value does not shrink it below fp32 resolution
+    of the sums.  relative_to="max" (pooled block logits, which straddle zero so that tau can
+    be arbitrarily close to 0): the bound is TIE_REL * max|candidate score|."""
     got = set(int(x) for x in np.asarray(got).tolist())
     ref = set(int(x) for x in np.asarray(ref).tolist())
     assert len(got) == len(ref), f"{what}: |gpu| = {len(got)} != |oracle| = {len(ref)}"
@@ -83,9 +90,15 @@ def near_tie_ok(got, ref, scores, cand=None, what=""):
         return 0
     sc = np.asarray(scores, np.float64).astype(np.float32).astype(np.float64)
     pool = sc if cand is None else sc[np.asarray(cand, bool)]
-    scale = float(np.max(np.abs(pool))) if pool.size else 1.0
+    top = float(np.max(np.abs(pool))) if pool.size else 0.0
     tau = float(min(sc[list(ref)])) if ref else 0.0
-    tol = TIE_REL * max(scale, 1e-30)
+    if relative_to == "tau":
+        tol = TIE_REL * max(abs(tau), 1e-3 * top)
+    elif relative_to == "max":
+        tol = TIE_REL * top
+    else:
+        raise ValueError(relative_to)
+    assert tol > 0.0, f"{what}: degenerate scores (all zero) cannot decide a tie"
     bad = [x for x in diff if abs(sc[x] - tau) > tol]
     assert not bad, f"{what}: {len(bad)} differing indices are not near-ties (tau={tau}, tol={tol}): {sorted(bad)[:8]}"
     return len(diff)
