@@ -347,9 +347,13 @@ class Plan:
 
     def attention_units(self):
         """(work units, key chunks) of msa_sparse_prefill for this plan."""
-        t = (_I64 * 2)()
+        return self.attention_work()[:2]
+
+    def attention_work(self):
+        """(work units, key chunks, unit bands) of msa_sparse_prefill for this plan."""
+        t = (_I64 * 3)()
         _check("msa_attention_units", _lib.msa_attention_units(self._h, ctypes.cast(t, _P)))
-        return int(t[0]), int(t[1])
+        return int(t[0]), int(t[1]), int(t[2])
 
     def selftest_timeout(self, ws, limit_us: int = 10000, stream=None):
         """Launch a bounded wait that runs out after limit_us; device_status then reports

@@ -52,6 +52,7 @@ struct AttnParams {
   uint32_t* next_item;     // work-unit counter, zero at launch
   int32_t n_units, n_kchunks, n_bands;
   uint32_t* chunk_done;    // per item: chunks whose state is in its accumulator (chunked keys)
+  uint32_t* band_done;     // per band: units finished (chunked keys)
   float* acc;              // accumulator slots [slot][128][ACC_ROW] (chunked keys)
   // index-based prefill (od not null): the Q rows of permuted classes are gathered from the
   // caller's Q by row index, and every output row goes to the caller's O at its original
@@ -98,7 +99,7 @@ struct __align__(1024) AttnSmem {
   uint64_t o_full[N_STREAMS], o_free[N_STREAMS];
   // work-item queue of each stream: ids taken from the global counter by the stream's TMA
   // thread, read by its MMA issuer and softmax warpgroup (-1 ends the stream)
-  int32_t iq[N_STREAMS][IQ_DEPTH][4];  // item, key chunk, accumulator slot
+  int32_t iq[N_STREAMS][IQ_DEPTH][4];  // item, key chunk, accumulator slot, band
   uint64_t iq_full[N_STREAMS][IQ_DEPTH], iq_empty[N_STREAMS][IQ_DEPTH];
   // softmax warpgroup handshakes around the accumulator of chunked items
   uint64_t acc_in[N_STREAMS], acc_out[N_STREAMS];
@@ -155,7 +156,7 @@ __device__ __forceinline__ bool load_item(const AttnParams& p, int item, ItemInf
 // the item's accumulator), last = no tiles of the item after this unit, total = the item's
 // tiles.  False: the item has no rows (every role skips it).
 struct UnitInfo {
-  int item, chunk, acc, k, total;
+  int item, chunk, acc, band, k, total;
   bool last;
 };
 
@@ -163,6 +164,7 @@ __device__ __forceinline__ bool load_unit(const AttnParams& p, const int32_t* e,
   u.item = e[0];
   u.chunk = e[1];
   u.acc = e[2];
+  u.band = e[3];
   if (!load_item(p, u.item, it)) return false;
   u.total = it.ntiles;
   u.k = 0;
@@ -178,12 +180,13 @@ __device__ __forceinline__ bool load_unit(const AttnParams& p, const int32_t* e,
   return true;
 }
 
-// Unit id -> (item, key chunk, accumulator slot).
-__device__ __forceinline__ void unit_entry(const AttnParams& p, int u, int32_t (&e)[3]) {
+// Unit id -> (item, key chunk, accumulator slot, band).
+__device__ __forceinline__ void unit_entry(const AttnParams& p, int u, int32_t (&e)[4]) {
   if (p.n_kchunks == 1) {
     e[0] = u;
     e[1] = 0;
     e[2] = -1;
+    e[3] = -1;
     return;
   }
   const UnitBand* b = reinterpret_cast<const UnitBand*>(p.ws + p.lay.bands);
@@ -198,6 +201,7 @@ __device__ __forceinline__ void unit_entry(const AttnParams& p, int u, int32_t (
   e[0] = bd.item0 + local % bd.n;
   e[1] = local / bd.n;
   e[2] = bd.acc0 + local % bd.n;
+  e[3] = lo;
 }
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
@@ -207,6 +211,42 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
 }
 __device__ __forceinline__ void st_release(uint32_t* a, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_release_add(uint32_t* a, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+
+// Accumulator slots of band b are those of bands b - 2, b - 4, ... (two buffers, alternate
+// bands).  Every unit counts itself finished in its band's counter once it no longer touches its
+// slot; a unit of band b >= 2 waits (bounded) until every unit of every earlier band of the same
+// parity has finished before its item's first write to the slot.  (Band b - 2 alone is not
+// enough: a band whose items all end in their first chunk with keys never writes a slot, so it
+// can finish while the band before it still uses the buffer.)  Earlier bands' units were all
+// handed out before any of band b, and a stream runs its units in the order it took them, so
+// the oldest unfinished unit never waits on a newer one.  known0 / known1: bands of even / odd
+// index below it are already known finished (a stream's bands only increase).
+__device__ __forceinline__ void band_unit_done(const AttnParams& p, const UnitInfo& u) {
+  if (p.band_done && u.band >= 0) red_release_add(p.band_done + u.band, 1u);
+}
+__device__ __forceinline__ bool band_wait_previous(const AttnParams& p, const UnitInfo& u, int& known0,
+                                                   int& known1, volatile int* abort) {
+  if (!p.band_done || u.band < 2) return true;
+  const bool odd = (u.band & 1) != 0;
+  const UnitBand* bands = reinterpret_cast<const UnitBand*>(p.ws + p.lay.bands);
+  const uint64_t t0 = global_ns();
+  for (int b = odd ? known1 : known0; b <= u.band - 2; b += 2) {
+    const uint32_t need = (uint32_t)bands[b].n * (uint32_t)p.n_kchunks;
+    while (ld_acquire(p.band_done + b) < need) {
+      if (*abort) return false;
+      if (global_ns() - t0 > 1000000000ull) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+  if (odd) known1 = u.band;
+  else known0 = u.band;
+  return true;
 }
 
 
@@ -433,7 +473,7 @@ __device__ __forceinline__ void mma_stream(const AttnParams& p, AttnSmem& sm, ui
   for (uint32_t qi = 0;; ++qi) {
     const uint32_t slot = qi % IQ_DEPTH;
     if (!mbar_wait(&sm.iq_full[s][slot], (qi / IQ_DEPTH) & 1, abort)) return;
-    const int32_t e[3] = {sm.iq[s][slot][0], sm.iq[s][slot][1], sm.iq[s][slot][2]};
+    const int32_t e[4] = {sm.iq[s][slot][0], sm.iq[s][slot][1], sm.iq[s][slot][2], sm.iq[s][slot][3]};
     mbar_arrive(&sm.iq_empty[s][slot]);
     if (e[0] < 0) break;
     ItemInfo it;
@@ -567,12 +607,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         int32_t e0 = -1;
         if (leader) {
           const int id = (int)atomicAdd(p.next_item, 1u);
-          int32_t e[3] = {-1, 0, -1};
+          int32_t e[4] = {-1, 0, -1, -1};
           if (id < p.n_units) unit_entry(p, id, e);
           e0 = e[0];
           sm.iq[s][slot][0] = e[0];
           sm.iq[s][slot][1] = e[1];
           sm.iq[s][slot][2] = e[2];
+          sm.iq[s][slot][3] = e[3];
           mbar_arrive(&sm.iq_full[s][slot]);
         }
         if constexpr (INDEXED) {
@@ -686,11 +727,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           }
         }
         if (uni(wd.expired(abort))) {
-          // let the copies already issued land before the CTA goes away
+          // let the copies already issued land before the CTA goes away: these waits ignore the
+          // CTA's abort flag (which is set by now) and give up only after their own limit
           if (leader) {
-            if (qt_iss) mbar_wait(&sm.q_full[s], (qt_iss - 1) & 1, abort, 100000000ull);
-            if (k_iss) mbar_wait(&sm.k_full[s], (k_iss - 1) & 1, abort, 100000000ull);
-            if (v_iss) mbar_wait(&sm.v_full[s], (v_iss - 1) & 1, abort, 100000000ull);
+            int drain_flag = 0;
+            if (qt_iss) mbar_wait(&sm.q_full[s], (qt_iss - 1) & 1, &drain_flag, 100000000ull);
+            if (k_iss) mbar_wait(&sm.k_full[s], (k_iss - 1) & 1, &drain_flag, 100000000ull);
+            if (v_iss) mbar_wait(&sm.v_full[s], (v_iss - 1) & 1, &drain_flag, 100000000ull);
           }
           wsync();
           break;
@@ -702,9 +745,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // warp 1: stream 0, warp 3: stream 1
     if (lane == 0) {
       mma_stream<INDEXED>(p, sm, tmem, warp >> 1, abort);
-      // wait for every MMA issued by this thread before the tensor memory is released
+      // wait for every MMA issued by this thread before the tensor memory is released; the wait
+      // ignores the CTA's abort flag (MMAs in flight must finish even after a timeout elsewhere)
+      // and gives up only after its own limit
       umma_commit(&sm.drain[warp >> 1]);
-      mbar_wait(&sm.drain[warp >> 1], 0, abort, 100000000ull);
+      int drain_flag = 0;
+      mbar_wait(&sm.drain[warp >> 1], 0, &drain_flag, 100000000ull);
     }
    }
   } else {
@@ -717,18 +763,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(p.ws + p.lay.op));
     const uint32_t* tiles = reinterpret_cast<const uint32_t*>(p.ws + p.lay.tiles);
     uint32_t s_count = 0, items_done = 0, acc_ins = 0, acc_outs = 0;
+    int bands_known0 = 0, bands_known1 = 1;  // unit bands of each parity known finished below these
     bool ok = true;
     for (uint32_t qi = 0; ok; ++qi) {
       const uint32_t slot = qi % IQ_DEPTH;
       if (!mbar_wait(&sm.iq_full[s][slot], (qi / IQ_DEPTH) & 1, abort)) break;
-      const int32_t e[3] = {sm.iq[s][slot][0], sm.iq[s][slot][1], sm.iq[s][slot][2]};
+      const int32_t e[4] = {sm.iq[s][slot][0], sm.iq[s][slot][1], sm.iq[s][slot][2], sm.iq[s][slot][3]};
       mbar_arrive(&sm.iq_empty[s][slot]);
       if (e[0] < 0) break;
       ItemInfo it;
       UnitInfo un;
-      if (!load_unit(p, e, it, un)) continue;
-      if (un.total > 0 && it.ntiles == 0) continue;  // no keys of this item in this chunk
-      if (un.total == 0 && un.chunk != 0) continue;  // an item without tiles is written once
+      // units that skip their work touch no accumulator slot: counted finished at once
+      if (!load_unit(p, e, it, un) ||
+          (un.total > 0 && it.ntiles == 0) ||  // no keys of this item in this chunk
+          (un.total == 0 && un.chunk != 0)) {  // an item without tiles is written once
+        if (t == 0) band_unit_done(p, un);
+        continue;
+      }
       const ClassStatic& cs = class_of(p, it.cls);
       const int r = it.row0 + t;
       RowCtx& rc = sm.rctx[threadIdx.x - 128];
@@ -748,6 +799,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           for (int i = 0; i < 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
           if (p.lse) p.lse[(size_t)it.head * p.L + rc.qpos] = -INFINITY;
         }
+        if (t == 0) band_unit_done(p, un);
         continue;
       }
 
@@ -881,6 +933,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       ++items_done;
       tc_fence_after();
       if (!un.last) {
+        // the item's first write to its slot: the earlier bands that used the slot must be done
+        // (each thread takes the counters with acquire itself; a continued item's slot was
+        // claimed by its first unit, in the same band)
+        if (!cont && !band_wait_previous(p, un, bands_known0, bands_known1, abort)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t oa[32];
@@ -904,10 +960,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           if (!mbar_wait(&sm.acc_out[s], acc_outs & 1, abort)) { ok = false; break; }
           __threadfence();
           st_release(p.chunk_done + un.item, (uint32_t)un.k + 1u);
+          band_unit_done(p, un);
         }
         ++acc_outs;
         continue;
       }
+      // the item's last unit: its slot was read (when continued) before its first P was handed
+      // to the tensor core, and this thread has seen the last P V of the unit, which needed
+      // every row's P: the slot is free
+      if (t == 0) band_unit_done(p, un);
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint4* dst = out_row();
 #pragma unroll
@@ -1060,6 +1121,7 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
   p.n_kchunks = dp.n_kchunks;
   p.n_bands = dp.n_bands;
   p.chunk_done = nullptr;
+  p.band_done = nullptr;
   p.acc = nullptr;
   p.qg = static_cast<const __nv_bfloat16*>(Q);
   p.qg_head = s.q_head;
@@ -1069,8 +1131,10 @@ cudaError_t launch_attention(const DevPlan& dp, const void* Q, const void* K, co
   p.od_row = s.o_row;
   if (dp.n_kchunks > 1) {
     p.chunk_done = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(ws + dp.lay.chunk_done));
+    p.band_done = p.chunk_done + dp.n_items;
     p.acc = reinterpret_cast<float*>(const_cast<uint8_t*>(ws + dp.lay.acc));
-    if (cudaError_t e = cudaMemsetAsync(p.chunk_done, 0, sizeof(uint32_t) * (size_t)dp.n_items, st)) return e;
+    if (cudaError_t e = cudaMemsetAsync(p.chunk_done, 0, sizeof(uint32_t) * ((size_t)dp.n_items + (size_t)dp.n_bands), st))
+      return e;
   }
   const size_t smem = sizeof(AttnSmem);
   static std::atomic<uint64_t> configured{0};

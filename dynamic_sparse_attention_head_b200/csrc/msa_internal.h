@@ -157,7 +157,8 @@ struct Layout {
   int64_t item_ntiles;       // int32 [n_items]
   int64_t bands;             // UnitBand [n_bands] (chunked keys only)
   int64_t cstart;            // int32 [n_items][n_kchunks + 1]: first tile of each key chunk (chunked keys only)
-  int64_t chunk_done;        // uint32 [n_items]: chunks of the item whose state is in its accumulator
+  int64_t chunk_done;        // uint32 [n_items]: chunks of the item whose state is in its accumulator,
+                             // then uint32 [n_bands]: finished units of each band
   int64_t acc;               // fp32 [n_acc][128][ACC_ROW]: per-item online-softmax state between chunks
   int64_t tiles;             // uint32 [total tile capacity]: (src << 28) | TILE_FULL? | first key row
   int64_t mask_pairs;        // uint64 [Hq]: allowed (query, key) pairs per head (msa_mask_pairs)

@@ -343,10 +343,16 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
     P->band_cap = 0;
     if (P->n_kchunks > 1) {
       // bands: runs of the plan order within one (KV head, key source, head kind) group and one
-      // range of 1024 slots, merged until each holds at least 2048 units, so that no more than
-      // two bands have units in flight (a stream holds at most five) and two accumulator
-      // buffers, used by alternate bands, suffice
-      constexpr int32_t BAND_SLOTS = 1024, MIN_UNITS = 2048;
+      // range of 1024 slots, merged until each holds at least 2048 units.  Alternate bands use
+      // two accumulator buffers; a unit of band b writes its item's slot only after every unit
+      // of band b - 2 (the previous user of the buffer) has finished (a per-band completion
+      // counter that the attention kernel waits on), so the two buffers are safe whatever the
+      // order in which the units complete.  The band size only decides how often that wait can
+      // stall.  MSA_ATTN_BAND_SLOTS and MSA_ATTN_MIN_BAND_UNITS (read here) override the two
+      // sizes, so that tests can make the bands tiny.
+      int32_t BAND_SLOTS = 1024, MIN_UNITS = 2048;
+      if (const char* env = std::getenv("MSA_ATTN_BAND_SLOTS")) BAND_SLOTS = std::max(1, std::atoi(env));
+      if (const char* env = std::getenv("MSA_ATTN_MIN_BAND_UNITS")) MIN_UNITS = std::max(1, std::atoi(env));
       auto key = [&](const WorkItem& w) {
         const ClassStatic& c = C[w.cls];
         return std::make_tuple(c.kvh, c.k_src, prob->heads[c.head].kind, w.slot / BAND_SLOTS);
@@ -476,7 +482,8 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   lay.item_ntiles = B.take(4 * (int64_t)P->items.size());
   if (P->n_kchunks > 1) {
     lay.cstart = B.take(4 * (int64_t)P->items.size() * (P->n_kchunks + 1));
-    lay.chunk_done = B.take(4 * (int64_t)P->items.size());
+    // chunk_done: uint32 [n_items] followed by the per-band completion counters [n_bands]
+    lay.chunk_done = B.take(4 * ((int64_t)P->items.size() + (int64_t)P->bands.size()));
     lay.acc = B.take(4 * 2 * (int64_t)P->band_cap * TILE * ACC_ROW, 1024);
   }
   lay.tiles = B.take(4 * P->total_tiles);
@@ -890,10 +897,11 @@ msa_status msa_device_status(const msa_plan* P, void* ws, void* stream) {
   return MSA_OK;
 }
 
-msa_status msa_attention_units(const msa_plan* P, int64_t out[2]) {
+msa_status msa_attention_units(const msa_plan* P, int64_t out[3]) {
   if (!P || !out) return MSA_ERR_INVALID_ARG;
   out[0] = P->n_units;
   out[1] = P->n_kchunks;
+  out[2] = (int64_t)P->bands.size();
   return MSA_OK;
 }
 

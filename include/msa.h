@@ -181,7 +181,12 @@ msa_status msa_permute(msa_plan* plan, const void* Q, const void* K, const void*
 msa_status msa_sparse_prefill(msa_plan* plan, const void* Q, const void* K, const void* V,
                               const msa_strides* strides, void* ws, size_t ws_bytes, float* lse, void* stream);
 
-/* Scatters the permuted output back to original token order into O (bf16, device). */
+/* Scatters the permuted output back to original token order into O (bf16, device):
+ * O[h][pos(r)] = O_perm[h][r] for every permuted row r.  The MMInference review page ("core
+ * discovery") requires the permutation to leave a head's output unchanged; this inverse
+ * gather is what makes the permuted computation return rows in the caller's order.  Output
+ * rows of identity (unpermuted) heads are copied as they are.  Layout and strides as for Q in
+ * msa_permute; asynchronous on `stream`. */
 msa_status msa_unpermute(msa_plan* plan, const void* ws, size_t ws_bytes, void* O, const msa_strides* strides,
                          void* stream);
 
@@ -226,13 +231,18 @@ msa_status msa_tile_stats(const msa_plan* plan, const void* ws, int64_t tiles[2]
 msa_status msa_mask_pairs(const msa_plan* plan, void* ws, int64_t* counts, void* stream);
 
 /* How msa_sparse_prefill divides its work (host only, no device access): out[0] = work units,
- * out[1] = key chunks.  When one head's K and V exceed about 96 MB (L > 192K tokens) the keys
- * are cut into chunks of 65536 (the environment variable MSA_ATTN_CHUNK_KEYS, a multiple of
- * 128, read at msa_plan_create, overrides the chunk size; 0 turns chunking off): the units of a
- * band of work items then run chunk by chunk so that the units in flight share one chunk of
- * K and V in L2, and a work item's online-softmax state passes from chunk to chunk through an
- * accumulator in the workspace.  The result does not depend on the chunking beyond rounding. */
-msa_status msa_attention_units(const msa_plan* plan, int64_t out[2]);
+ * out[1] = key chunks, out[2] = unit bands (0 when the keys are not chunked).  When one head's
+ * K and V exceed about 96 MB (L > 192K tokens) the keys are cut into chunks of 65536 (the
+ * environment variable MSA_ATTN_CHUNK_KEYS, a multiple of 128, read at msa_plan_create,
+ * overrides the chunk size; 0 turns chunking off): the units of a band of work items then run
+ * chunk by chunk so that the units in flight share one chunk of K and V in L2, and a work
+ * item's online-softmax state passes from chunk to chunk through an accumulator slot in the
+ * workspace.  Alternate bands share two sets of slots; a unit writes a slot only after every
+ * unit of the band that used it before has finished.  Bands are runs of up to 1024 query-tile
+ * slots of one KV head, key source and head kind, merged up to at least 2048 units
+ * (MSA_ATTN_BAND_SLOTS and MSA_ATTN_MIN_BAND_UNITS, read at msa_plan_create, override the two
+ * numbers).  The result does not depend on the chunking or the bands beyond rounding. */
+msa_status msa_attention_units(const msa_plan* plan, int64_t out[3]);
 
 /* Dumps the work list of head `head` for tests: for each of its 128-query work items the
  * query positions covered (-1 for padding) and, for every executed tile, its key source
@@ -263,7 +273,9 @@ const char* msa_status_string(msa_status status);
 /* ---- allocation-free variant ----
  *
  * Vertical-slash index estimation of ONE query head (the vertical and slash lines of its last
- * 64 queries, exactly as msa_estimate computes them for a vertical-slash head) for callers
+ * 64 queries, by the rules msa_estimate applies to a vertical-slash head; its sums may be
+ * rounded in another order, so at near-ties its lines may differ from msa_estimate's within
+ * the tolerance both keep against an exact computation) for callers
  * that cannot allocate device memory or provide a workspace: code running inside another
  * framework's memory manager, or serving loops where cudaMalloc and its implicit device
  * synchronisation are not allowed.  This call has no counterpart in the method's description;

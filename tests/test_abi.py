@@ -92,6 +92,27 @@ def test_attention_units_chunking_rule(monkeypatch):
     assert chunks == 1
 
 
+def test_unit_band_overrides(monkeypatch):
+    """Unit bands exist only over chunked keys; the band-size overrides apply at plan creation
+    and only change how the units are grouped, not how many there are."""
+    import dynamic_sparse_attention_head_b200 as msa
+    import workload
+    p = workload.llama3_8b_text(L=2048)
+    monkeypatch.delenv("MSA_ATTN_BAND_SLOTS", raising=False)
+    monkeypatch.delenv("MSA_ATTN_MIN_BAND_UNITS", raising=False)
+    monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", "0")
+    assert msa.Plan(p).attention_work()[2] == 0
+    monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", "256")
+    units, chunks, bands = msa.Plan(p).attention_work()
+    assert chunks == 8 and bands >= 1
+    monkeypatch.setenv("MSA_ATTN_BAND_SLOTS", "1")
+    monkeypatch.setenv("MSA_ATTN_MIN_BAND_UNITS", "1")
+    units2, chunks2, bands2 = msa.Plan(p).attention_work()
+    assert (units2, chunks2) == (units, chunks) and bands2 > bands
+    items = units // chunks
+    assert bands2 <= items
+
+
 def test_workspace_size_and_state_checks_come_before_any_device_access():
     """The size, alignment and call-order checks of the calls return before anything touches
     device memory, so they are exercised here with placeholder addresses (never dereferenced)."""

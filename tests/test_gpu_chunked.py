@@ -76,3 +76,30 @@ def test_chunked_mixed_layer_equals_unchunked(monkeypatch):
     fin = np.isfinite(l0)
     assert np.array_equal(fin, np.isfinite(l1))
     np.testing.assert_allclose(l1[fin], l0[fin], atol=1e-3, rtol=1e-4)
+
+
+@pytest.mark.parametrize("band_slots,min_units", [(1, 1), (2, 16), (1, 40)])
+def test_tiny_bands_match_oracle_on_all_rows(band_slots, min_units, monkeypatch):
+    """Many small unit bands (MSA_ATTN_BAND_SLOTS / MSA_ATTN_MIN_BAND_UNITS) over small key
+    chunks, on a layer whose items are long and short (every head kind, one KV head): alternate
+    bands share two sets of accumulator slots, so every slot is reused many times while units
+    of earlier bands may still be running.  All rows against the oracle, and three launches
+    bit-identical (a unit that wrote into a slot still in use would make them differ)."""
+    p = mixed_problem()
+    Q, K, V = make_inputs(p, seed=12)
+    idx = oracle.estimate(p, Q, K)
+    monkeypatch.setenv("MSA_ATTN_BAND_SLOTS", str(band_slots))
+    monkeypatch.setenv("MSA_ATTN_MIN_BAND_UNITS", str(min_units))
+    monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", "128")
+    units, chunks, bands = msa.Plan(p).attention_work()
+    assert chunks == (p.L + 127) // 128 and bands >= 8, (units, chunks, bands)
+    runs = [_run(p, Q, K, V, idx, monkeypatch, 128) for _ in range(3)]
+    O, lse = runs[0]
+    for O2, l2 in runs[1:]:
+        assert np.array_equal(O2, O) and np.array_equal(l2, lse, equal_nan=True)
+    Oref, lref = oracle.attention(p, Q, K, V, idx)
+    for h in range(p.Hq):
+        compare_outputs(O[h], Oref[h], f"head {h} bands {bands}")
+        fin = np.isfinite(lref[h])
+        assert np.array_equal(fin, np.isfinite(lse[h])), f"head {h}: empty rows differ"
+        np.testing.assert_allclose(lse[h][fin], lref[h][fin], atol=2e-3, rtol=1e-3)
