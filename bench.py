@@ -32,6 +32,9 @@ import workload  # noqa: E402
 
 METRIC = "sparse-prefill attention ms/layer + effective TFLOP/s at 128K and 1M tokens"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's B200 dense bf16 tensor peak (half of the 2:4-sparse datasheet figure): context only,
+# beside the measured peaks that the fractions are taken against
+DATASHEET_BF16_DENSE_TFLOPS = 2250.0
 
 
 def workloads():
@@ -127,13 +130,22 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # CPU oracle on a bounded sample (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------------------
-def oracle_sample(p, Q, K, V, rows_per_head=32, seed=0):
+def sample_rows(L, n, seed):
+    """n query rows stratified over [0, L): one seeded uniform row per stratum of L / n rows, so
+    that the sample covers the whole causal range evenly (masked-attention time per row grows
+    with the row's position)."""
+    rng = np.random.default_rng(seed)
+    n = max(1, min(n, L))
+    edges = np.linspace(0, L, n + 1).astype(np.int64)
+    return np.array([rng.integers(lo, hi) for lo, hi in zip(edges[:-1], edges[1:]) if hi > lo], np.int64)
+
+
+def oracle_sample(p, Q, K, V, rows_per_head=4096, seed=0):
     """Times the oracle on one head of each kind: its full index estimation plus masked
-    attention for `rows_per_head` uniformly sampled query rows, the attention time scaled by
-    L / rows (attention time is proportional to rows on a uniform sample).  Returns per-kind
+    attention of `rows_per_head` stratified seeded rows, the attention time scaled by
+    L / rows (an unbiased estimate of the whole head's attention time).  Returns per-kind
     seconds for one head and the sampled heads."""
     import oracle
-    rng = np.random.default_rng(seed)
     heads = {}
     for h, hd in enumerate(p.heads):
         heads.setdefault(hd.kind, h)
@@ -142,10 +154,11 @@ def oracle_sample(p, Q, K, V, rows_per_head=32, seed=0):
         t0 = time.perf_counter()
         idx = oracle.estimate_head(p, h, Q, K)
         t1 = time.perf_counter()
-        rows = np.sort(rng.choice(p.L, size=min(rows_per_head, p.L), replace=False))
+        rows = sample_rows(p.L, rows_per_head, seed * 1000 + h)
         oracle.attention_head(p, h, Q, K, V, idx, rows)
         t2 = time.perf_counter()
-        per_kind[kind] = {"head": h, "est_s": t1 - t0, "attn_s": (t2 - t1) * p.L / len(rows), "idx": idx}
+        per_kind[kind] = {"head": h, "est_s": t1 - t0, "attn_s": (t2 - t1) * p.L / len(rows), "idx": idx,
+                          "rows": len(rows), "sampled_s": t2 - t0}
     return per_kind
 
 
@@ -211,14 +224,36 @@ def recorded_traffic(workload_name):
     return ent.get("dram_bytes_per_launch")
 
 
-def run_ours(args, rank, world, local_rank):
+SECONDARY = {"qwen2-7b-video-128k": "longvila-1m"}  # the metric is quoted at 128K and at 1M
+
+
+def per_kind_stats(p, tiles_per_head, pairs_per_head):
+    """Executed density (executed block FLOPs / dense causal FLOPs) and mask density (allowed
+    pairs / dense causal pairs) of each head kind of the layer."""
+    dense_head = 2 * p.d * p.L * (p.L + 1)
+    out = {}
+    for kind in dict.fromkeys(h.kind for h in p.heads):
+        hs = [h for h, hd in enumerate(p.heads) if hd.kind == kind]
+        ex = sum(4 * 128 ** 3 * int(tiles_per_head[h]) for h in hs)
+        us = sum(4 * p.d * int(pairs_per_head[h]) for h in hs)
+        out[kind] = {"heads": len(hs), "executed_density": ex / (dense_head * len(hs)),
+                     "mask_density": us / (dense_head * len(hs)),
+                     "useful_over_executed": us / ex if ex else None}
+    return out
+
+
+def measure_layer(args, name, rank, world, local_rank, steps, warmup, with_e2e, with_cpu, with_dense):
+    """Times `steps` steps of the named layer after `warmup` untimed ones (inputs resident) and
+    returns the measurement as a dict (the JSON line's fields except the header)."""
+    import dataclasses
+
     import torch
     import dynamic_sparse_attention_head_b200 as msa
     import torch.distributed as dist
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    p = workloads()[args.workload]()
+    p = workloads()[name]()
     Qh, Kh, Vh = make_host_inputs(p, seed=rank)
 
     def dev_copy(x):
@@ -265,18 +300,20 @@ def run_ours(args, rank, world, local_rank):
             events[1].record(stream)
         prefill(q, k, v, o, events)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     status = plan.device_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
     tiles, items = plan.tile_stats(ws)
+    tiles_head = plan.tile_stats_heads(ws)
     exec_flops = msa.executed_flops(tiles)
     # allowed (query, key) pairs under the masks, counted on the device before the timed region
-    useful_flops = 4 * p.d * int(plan.mask_pairs(ws).sum())
+    pairs_head = plan.mask_pairs(ws)
+    useful_flops = 4 * p.d * int(pairs_head.sum())
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -289,7 +326,7 @@ def run_ours(args, rank, world, local_rank):
     n0 = msa.kernel_launches()
     with ClockSampler(uuid) as clk:
         start.record(stream)
-        for s in range(args.steps):
+        for s in range(steps):
             step(evs[s])
         end.record(stream)
         torch.cuda.synchronize()
@@ -300,8 +337,8 @@ def run_ours(args, rank, world, local_rank):
     stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # ms
     # max over ranks of the timed region; sum of executed FLOPs over ranks
     total_ms, job_flops = job_totals(total_ms, exec_flops, world, dev)
-    ms_step = total_ms / args.steps
-    value = job_flops * args.steps / (total_ms * 1e-3) / 1e12
+    ms_step = total_ms / steps
+    value = job_flops * steps / (total_ms * 1e-3) / 1e12
 
     # end to end through the public API with host buffers: every step copies its Q/K/V from
     # pinned host memory, runs the path and reads its O back to pinned host memory.  The copies
@@ -309,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
     # H2D copy of step s+1 and the D2H copy of step s-1 run on copy streams while step s
     # computes; the timed region spans the first H2D copy to the last D2H copy.
     e2e = None
-    if not args.no_e2e:
+    if with_e2e:
         qp = torch.from_numpy(Qh).view(torch.bfloat16).pin_memory()
         kp = torch.from_numpy(Kh).view(torch.bfloat16).pin_memory()
         vp = torch.from_numpy(Vh).view(torch.bfloat16).pin_memory()
@@ -348,64 +385,116 @@ def run_ours(args, rank, world, local_rank):
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
         h2d.wait_event(s0)
-        run_e2e(args.steps)
+        run_e2e(steps)
         stream.wait_stream(d2h)
         s1.record(stream)
         torch.cuda.synchronize()
         e2e_ms, _ = job_totals(s0.elapsed_time(s1), 0.0, world, dev)
         bi = (Qh.nbytes + Kh.nbytes + Vh.nbytes)
         bo = int(np.prod(o.shape)) * 2
-        e2e = {"value": job_flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / args.steps,
+        e2e = {"value": job_flops * steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms / steps,
                "copies": "pipelined across steps (two device buffer sets, H2D and D2H streams)"}
+        del bufs, qp, kp, vp, ohost
 
     pk, pk_src = peaks()
     attn_ms = float(stage[:, 2].mean())
     achieved = exec_flops / (attn_ms * 1e-3) / 1e12
     peak_sus = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    traffic = recorded_traffic(args.workload + ("+indexed" if args.indexed else ""))
+    traffic = recorded_traffic(name + ("+indexed" if args.indexed else ""))
     roofline = {"kernel": "msa_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": peak_sus,
                 "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
                 "peak_source": f"{pk_src} bf16_tflops_sustained (kernel inside a long step)",
                 "frac_of_burst_peak": achieved / peak_burst,
+                "frac_of_datasheet_dense_peak": achieved / DATASHEET_BF16_DENSE_TFLOPS,
                 "flops_per_launch": exec_flops, "ms_per_launch": attn_ms,
                 **({"timed": "msa_sparse_prefill_indexed: the key gathers (a few % of its bytes, "
                              "under 0.2 % of its time) and the attention kernel"} if args.indexed else {})}
 
+    # the same layer with every head dense, through the same kernel, timed once outside the
+    # timed region: what the sparse index saves against dense attention on this hardware
+    dense = None
+    if with_dense and not args.indexed:
+        pd_ = dataclasses.replace(p, heads=[workload.Head("dense")] * p.Hq)
+        plan_d = msa.Plan(pd_)
+        ws_d = plan_d.alloc_workspace()
+        plan_d.estimate(q, k, ws_d)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for rep in range(2):  # one untimed pass, then the timed one
+            plan_d.permute(q, k, v, ws_d)
+            e0.record(stream)
+            plan_d.sparse_prefill(q, k, v, ws_d)
+            e1.record(stream)
+            plan_d.unpermute(ws_d, o)
+            torch.cuda.synchronize()
+        assert plan_d.device_status(ws_d) == 0
+        dense_ms = e0.elapsed_time(e1)
+        dtiles, _ = plan_d.tile_stats(ws_d)
+        dense = {"attention_ms": dense_ms, "executed_flops": msa.executed_flops(dtiles),
+                 "tflops": msa.executed_flops(dtiles) / (dense_ms * 1e-3) / 1e12,
+                 "speedup_vs_dense_same_kernel": dense_ms / attn_ms,
+                 "layer_speedup_vs_dense_attention": dense_ms / ms_step}
+        del ws_d, plan_d
+        torch.cuda.empty_cache()
+
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if with_cpu and rank == 0 and world == 1:
         per_kind = oracle_sample(p, Qh, Kh, Vh, rows_per_head=args.cpu_rows)
         layer_s = oracle_layer_seconds(p, per_kind)
+        rows = max(v_["rows"] for v_ in per_kind.values())
         cpu = {"value": exec_flops / layer_s / 1e12, "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
-               "ms_per_layer": layer_s * 1e3,
+               "ms_per_layer": layer_s * 1e3, "extrapolated": True, "sampled_rows_per_head": rows,
+               "sampled_seconds": sum(v_["sampled_s"] for v_ in per_kind.values()),
                "sample": (f"oracle on one head of each kind ({', '.join(per_kind)}): full index estimation + "
-                          f"masked attention of {args.cpu_rows} uniformly sampled rows scaled to L rows; "
-                          f"layer time = sum over heads of their kind's time; value = this layer's executed "
-                          f"block FLOPs / that time")}
+                          f"masked attention of {rows} stratified seeded rows, scaled to L rows; "
+                          f"layer time = sum over heads of their kind's time (extrapolated); value = this "
+                          f"layer's executed block FLOPs / that time")}
 
+    sm = clk.summary()
+    dcf = dense_causal_flops(p)
+    return {
+        "value": value, "ms_per_step": ms_step, "ms_per_layer": ms_step, "steps": steps, "warmup": warmup,
+        "config": {"workload": name, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
+                   "heads": kind_summary(p), "parallelism": f"independent layer per rank x{world}",
+                   "l2": "inputs larger than L2 (no flush)" if (Qh.nbytes > 126e6) else "inputs smaller than L2",
+                   "seed": "rank", **({"estimate_every": args.estimate_every} if args.estimate_every > 1 else {}),
+                   **({"path": "index-based (Q rows gathered in the attention kernel, O written at "
+                               "original positions)"} if args.indexed else {})},
+        "stages_ms": {"estimate": float(stage[:, 0].mean()), "permute": float(stage[:, 1].mean()),
+                      "attention": attn_ms, "unpermute": float(stage[:, 3].mean())},
+        "executed_tiles": tiles, "work_items": items, "executed_flops": exec_flops,
+        "useful_flops": useful_flops, "dense_causal_flops": dcf,
+        "mask_density": useful_flops / dcf, "executed_density": exec_flops / dcf,
+        "useful_over_executed": useful_flops / exec_flops if exec_flops else None,
+        "dense_flops_avoided": dcf - useful_flops,
+        "per_kind": per_kind_stats(p, tiles_head, pairs_head),
+        "dense_same_kernel": dense,
+        "attn_tflops": achieved,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+        "clocks": sm,
+    }
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    main = measure_layer(args, args.workload, rank, world, local_rank, args.steps, args.warmup,
+                         with_e2e=not args.no_e2e, with_cpu=not args.no_cpu_baseline,
+                         with_dense=not args.no_dense)
+    torch.cuda.empty_cache()
+    second = None
+    sec_name = SECONDARY.get(args.workload) if not args.no_secondary else None
+    if sec_name:
+        second = measure_layer(args, sec_name, rank, world, local_rank, args.secondary_steps,
+                               max(3, min(args.warmup, 3)), with_e2e=not args.no_e2e, with_cpu=False,
+                               with_dense=not args.no_dense)
+        second = {"metric": METRIC, "unit": "TFLOP/s", **second}
     if rank == 0:
-        sm = clk.summary()
-        line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "ms_per_layer": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
-                       "heads": kind_summary(p), "parallelism": f"independent layer per rank x{world}",
-                       "l2": "inputs larger than L2 (no flush)" if (Qh.nbytes > 126e6) else "inputs smaller than L2",
-                       "seed": "rank", **({"estimate_every": args.estimate_every} if args.estimate_every > 1 else {}),
-                       **({"path": "index-based (Q rows gathered in the attention kernel, O written at "
-                                   "original positions)"} if args.indexed else {})},
-            "stages_ms": {"estimate": float(stage[:, 0].mean()), "permute": float(stage[:, 1].mean()),
-                          "attention": attn_ms, "unpermute": float(stage[:, 3].mean())},
-            "executed_tiles": tiles, "work_items": items, "executed_flops": exec_flops,
-            "useful_flops": useful_flops, "dense_causal_flops": dense_causal_flops(p),
-            "mask_density": useful_flops / dense_causal_flops(p),
-            "dense_flops_avoided": dense_causal_flops(p) - useful_flops,
-            "attn_tflops": achieved,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
-            "clocks": sm,
-        }
+        line = {"metric": METRIC, "value": main.pop("value"), "unit": "TFLOP/s", "n_gpus": world,
+                "steps": main.pop("steps"), "warmup": main.pop("warmup"), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", **main}
+        if second is not None:
+            line["secondary"] = second
         print(json.dumps(line), flush=True)
 
 
@@ -485,16 +574,22 @@ def run_reference(args, rank, world):
     flops = executed_flops_for(p, per_kind)
     layer_s = float(np.mean(times))
     value = flops / layer_s / 1e12 if flops else None
+    rows = max(v_["rows"] for v_ in per_kind.values())
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": layer_s * 1e3, "ms_per_layer": layer_s * 1e3,
+            "extrapolated": True, "sampled_rows_per_head": rows,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
+            "value_basis": ("the layer's executed block FLOPs (the unit of the metric, counted once, untimed, "
+                            "from the oracle's own index sets) / the oracle's extrapolated layer time, so "
+                            "that the ratio of the two arms' values is the ratio of their layer times"),
             "config": {"workload": args.workload, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
                        "heads": kind_summary(p)},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
-                             "sample": (f"per step: oracle on one head of each kind, full estimation + "
-                                        f"{args.cpu_rows} sampled rows of masked attention scaled to L rows; "
-                                        f"layer time summed over heads by kind")},
+                             "extrapolated": True, "sampled_rows_per_head": rows,
+                             "sample": (f"per step: oracle on one head of each kind, full index estimation + "
+                                        f"masked attention of {rows} stratified seeded rows, scaled to L rows; "
+                                        f"layer time summed over heads by kind (extrapolated)")},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -526,7 +621,13 @@ def main():
     ap.add_argument("--workload", default="qwen2-7b-video-128k", choices=sorted(workloads()))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=32)
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip timing the all-dense layer through the same kernel (outside the timed region)")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the second line of the metric (the 1M layer after the 128K one)")
+    ap.add_argument("--secondary-steps", type=int, default=3)
+    ap.add_argument("--cpu-rows", type=int, default=4096,
+                    help="query rows per sampled head in the oracle's timed sample")
     ap.add_argument("--sweep", action="store_true", help="budget sweep table instead of the benchmark line")
     ap.add_argument("--estimate-every", type=int, default=1,
                     help="estimate indices on every K-th layer only and reuse them in between (index "

@@ -75,6 +75,7 @@ def _load():
         "msa_read_indices": ([_P, _P, _I32, _P, ctypes.POINTER(_I64), _P], _I32),
         "msa_read_tiles": ([_P, _P, _I32, _P, ctypes.POINTER(_I64), _P], _I32),
         "msa_tile_stats": ([_P, _P, _P, _P], _I32),
+        "msa_tile_stats_heads": ([_P, _P, _P, _P], _I32),
         "msa_attention_units": ([_P, _P], _I32),
         "msa_mask_pairs": ([_P, _P, _P, _P], _I32),
         "msa_selftest_timeout": ([_P, _P, ctypes.c_uint32, _P], _I32),
@@ -94,7 +95,7 @@ _lib = _load()
 EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_workspace_bytes_indexed",
            "msa_sparse_prefill_indexed", "msa_estimate", "msa_set_indices",
            "msa_permute", "msa_sparse_prefill", "msa_unpermute", "msa_read_indices", "msa_read_tiles",
-           "msa_tile_stats", "msa_attention_units", "msa_mask_pairs", "msa_selftest_timeout", "msa_device_status", "msa_status_string",
+           "msa_tile_stats", "msa_tile_stats_heads", "msa_attention_units", "msa_mask_pairs", "msa_selftest_timeout", "msa_device_status", "msa_status_string",
            "msa_kernel_launches", "msa_vslash_estimate_static")
 
 
@@ -336,6 +337,14 @@ class Plan:
         t = (_I64 * 2)()
         _check("msa_tile_stats", _lib.msa_tile_stats(self._h, ws.data_ptr(), ctypes.cast(t, _P), _stream_ptr(stream)))
         return int(t[0]), int(t[1])
+
+    def tile_stats_heads(self, ws, stream=None):
+        """Executed tiles of each query head (int64 [Hq])."""
+        import numpy as np
+        c = np.zeros(self.problem.Hq, np.int64)
+        _check("msa_tile_stats_heads", _lib.msa_tile_stats_heads(self._h, ws.data_ptr(), c.ctypes.data_as(_P),
+                                                                 _stream_ptr(stream)))
+        return c
 
     def mask_pairs(self, ws, stream=None):
         """Allowed (query, key) pairs per query head under the current masks (int64 [Hq]);

@@ -28,7 +28,8 @@ struct DevPlan {
   int64_t n_text;      // text tokens (they lead the modality-grouped order)
   int32_t tb_words;    // unit-bitmap words per tile-builder warp
   int32_t max_chunks;  // most key chunks of any row set
-  int32_t sacc_n;      // slash accumulator entries the second estimation pass needs per block
+  int32_t n_lqtiles;   // tiles of the last-query sweep (pairs of row sets)
+  int32_t lq_ring;     // slash ring entries per row set in the second sweep pass (power of two)
   float scale;
   const int32_t* class_kind;  // host copy: kind of each class
 };
@@ -49,7 +50,15 @@ void count_launches(int n);
 // layout of modalities / ranks / modality-grouped order from the segment table
 cudaError_t launch_layout(const DevPlan& dp, cudaStream_t st);
 // last-64-query sweeps (two passes) and top-k jobs
+// Modality-grouped copy of K (text rows, then video rows) for the 2D-boundary heads.
+cudaError_t launch_group_k(const DevPlan& dp, const void* K, const msa_strides& s, cudaStream_t st);
 cudaError_t launch_lastq(const DevPlan& dp, const void* Q, const void* K, const msa_strides& s, cudaStream_t st);
+// Slash-ring entries per row set the second sweep pass needs for row sets spanning max_span
+// coordinates (a power of two), and the shared memory of each pass.
+int lastq_ring_entries(int32_t max_span);
+// Key chunk of the sweep for tiles reaching the given keys (one CTA per tile and chunk).
+int32_t lastq_pick_chunk(const int32_t* tile_key_hi, int n_tiles);
+size_t lastq_smem_bytes(int pass, int ring);
 cudaError_t launch_topk_jobs(const DevPlan& dp, cudaStream_t st);
 // block-sparse pooled estimation
 cudaError_t launch_block_estimate(const DevPlan& dp, const void* Q, const void* K, const msa_strides& s,

@@ -116,6 +116,16 @@ struct RowSet {
   int32_t n_chunks, chunk;   // key chunks of the sweep
 };
 
+// One tile of the last-query sweep: up to two row sets of one KV head and key source, stacked
+// as the 128 rows (row set 0: rows 0-63, row set 1: rows 64-127) of one tensor-core tile, so
+// that their logits come from one MMA per key block and K is streamed once for both.
+struct LqTile {
+  int32_t rs[2];             // row set indices (rs[1] = -1: rows 64-127 are padding)
+  int32_t kvh, k_src;
+  int32_t key_hi;            // keys [0, key_hi) of the source (the larger of the two row sets')
+  int32_t n_chunks;          // key chunks (the larger of the two row sets')
+};
+
 struct TopkJob {
   int64_t score_off;         // fp32 scores
   int32_t lo, hi;            // candidate index range [lo, hi)
@@ -150,6 +160,7 @@ struct Layout {
   int64_t classes;           // ClassStatic [n_classes]
   int64_t heads;             // HeadStatic [Hq]
   int64_t rowsets;           // RowSet [n_rowsets]
+  int64_t lq_tiles;          // LqTile [n_lqtiles]
   int64_t jobs;              // TopkJob [n_jobs]
   int64_t items;             // WorkItem [n_items]
   int64_t segs;              // int32 [n_segments][3] start, len, modality

@@ -8,7 +8,8 @@
 // the inputs (Q and K of the head) and the outputs (the two index lists and their counts).
 //
 // It runs the same kernels as msa_estimate (two-pass last-64-query sweep, deterministic
-// top-k) on a one-head plan whose workspace is the static array.
+// top-k) with the same key chunking, on a one-head plan whose workspace is the static array,
+// so its lines are those msa_estimate finds for a one-head vertical-slash plan.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -23,10 +24,10 @@ namespace msa {
 namespace {
 
 constexpr int64_t NOALLOC_MAX_L = 65536;
-constexpr int64_t NOALLOC_CHUNK = 1024;
-// header + tables (1 KB) + v, s (4 B per key each) + chunk partials + row stats + the two lists
-constexpr size_t NOALLOC_BYTES = 4096 + 2 * 4 * NOALLOC_MAX_L + (NOALLOC_MAX_L / NOALLOC_CHUNK) * LASTQ * 2 * 4 +
-                                 LASTQ * 2 * 4 + 2 * 4 * NOALLOC_MAX_L + 256;
+constexpr int64_t NOALLOC_MIN_CHUNK = 256;  // the sweep's smallest key chunk
+// header + tables (2 KB) + v, s (4 B per key each) + chunk partials + row stats + the two lists
+constexpr size_t NOALLOC_BYTES = 4096 + 2 * 4 * NOALLOC_MAX_L + (NOALLOC_MAX_L / NOALLOC_MIN_CHUNK) * LASTQ * 2 * 4 +
+                                 LASTQ * 2 * 4 + 2 * 4 * NOALLOC_MAX_L + 512;
 
 __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
 
@@ -54,6 +55,7 @@ inline int64_t up256(int64_t x) { return (x + 255) / 256 * 256; }
 
 struct Tables {
   RowSet rs;
+  LqTile tile;
   TopkJob jv, js;
 };
 
@@ -61,6 +63,7 @@ struct Tables {
 __global__ void noalloc_setup_kernel(uint8_t* ws, Layout lay, Tables t) {
   if (threadIdx.x == 0 && blockIdx.x == 0) {
     *reinterpret_cast<RowSet*>(ws + lay.rowsets) = t.rs;
+    *reinterpret_cast<LqTile*>(ws + lay.lq_tiles) = t.tile;
     reinterpret_cast<TopkJob*>(ws + lay.jobs)[0] = t.jv;
     reinterpret_cast<TopkJob*>(ws + lay.jobs)[1] = t.js;
     reinterpret_cast<uint32_t*>(ws + lay.header)[0] = 0u;
@@ -105,14 +108,18 @@ extern "C" msa_status msa_vslash_estimate_static(const void* Q, const void* K, i
   if (scratch_address(&scratch) != cudaSuccess) return MSA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // one-head layout inside the scratch
-  const int32_t n_chunks = (int32_t)((L + NOALLOC_CHUNK - 1) / NOALLOC_CHUNK);
+  // one-head layout inside the scratch; the sweep's key chunk by msa_estimate's rule
+  const int32_t key_hi = (int32_t)L;
+  const int32_t chunk = lastq_pick_chunk(&key_hi, 1);
+  const int32_t n_chunks = (int32_t)((L + chunk - 1) / chunk);
   Layout lay{};
   int64_t off = 0;
   lay.header = off;
   off += 256;
   lay.rowsets = off;
   off = up256(off + (int64_t)sizeof(RowSet));
+  lay.lq_tiles = off;
+  off = up256(off + (int64_t)sizeof(LqTile));
   lay.jobs = off;
   off = up256(off + 2 * (int64_t)sizeof(TopkJob));
   const int64_t cnt_off = off;
@@ -146,8 +153,14 @@ extern "C" msa_status msa_vslash_estimate_static(const void* Q, const void* K, i
   r.s_off = s_off;
   r.mz_off = mz_off;
   r.stat_off = stat_off;
-  r.chunk = (int32_t)NOALLOC_CHUNK;
+  r.chunk = chunk;
   r.n_chunks = n_chunks;
+  t.tile.rs[0] = 0;
+  t.tile.rs[1] = -1;
+  t.tile.kvh = 0;
+  t.tile.k_src = SRC_K;
+  t.tile.key_hi = (int32_t)L;
+  t.tile.n_chunks = n_chunks;
   t.jv.score_off = v_off;
   t.jv.lo = 0;
   t.jv.hi = (int32_t)L;
@@ -170,7 +183,8 @@ extern "C" msa_status msa_vslash_estimate_static(const void* Q, const void* K, i
   dp.n_rowsets = 1;
   dp.n_jobs = 2;
   dp.max_chunks = n_chunks;
-  dp.sacc_n = (LASTQ - 1) + (int32_t)NOALLOC_CHUNK + 64 + 64;  // consecutive rows: span 63
+  dp.n_lqtiles = 1;
+  dp.lq_ring = lastq_ring_entries(LASTQ - 1);  // consecutive rows: span 63
   dp.scale = scale;
   dp.has2d = 0;
   msa_strides s{};

@@ -36,6 +36,7 @@ struct msa_plan {
   std::vector<ClassStatic> classes;
   std::vector<HeadStatic> hs;
   std::vector<RowSet> rowsets;
+  std::vector<LqTile> lqtiles;
   std::vector<TopkJob> jobs;
   std::vector<WorkItem> items;
   std::vector<UnitBand> bands;
@@ -441,19 +442,35 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
       default: break;
     }
   }
-  // Key chunks of the estimation passes (one block each): 1024 keys, halved down to 256 while
-  // the passes would launch fewer than eight blocks per SM.
-  int32_t chunk = 1024;
+  // Tiles of the last-query sweep: row sets of one KV head and key source, paired in the order
+  // they were made (a head's own row sets first), two per 128-row tensor-core tile.
+  std::vector<LqTile>& LT = P->lqtiles;
+  LT.clear();
   {
-    int64_t blocks = 0;
-    for (const auto& r : RS) blocks += (r.key_hi + chunk - 1) / chunk;
-    while (chunk > 256 && blocks < 8LL * sm_count()) {
-      chunk /= 2;
-      blocks = 0;
-      for (const auto& r : RS) blocks += (r.key_hi + chunk - 1) / chunk;
+    std::vector<bool> used(RS.size(), false);
+    for (size_t i = 0; i < RS.size(); ++i) {
+      if (used[i]) continue;
+      used[i] = true;
+      LqTile t{};
+      t.rs[0] = (int32_t)i;
+      t.rs[1] = -1;
+      t.kvh = RS[i].kvh;
+      t.k_src = RS[i].k_src;
+      for (size_t j = i + 1; j < RS.size(); ++j)
+        if (!used[j] && RS[j].kvh == t.kvh && RS[j].k_src == t.k_src) {
+          used[j] = true;
+          t.rs[1] = (int32_t)j;
+          break;
+        }
+      LT.push_back(t);
     }
   }
-  int32_t sacc_n = 0;
+  // key chunks of the sweep (one CTA per tile and chunk)
+  std::vector<int32_t> tile_hi;
+  for (const auto& t : LT)
+    tile_hi.push_back(t.rs[1] >= 0 ? std::max(RS[t.rs[0]].key_hi, RS[t.rs[1]].key_hi) : RS[t.rs[0]].key_hi);
+  const int32_t chunk = lastq_pick_chunk(tile_hi.data(), (int)tile_hi.size());
+  int32_t max_span = 0;
   for (auto& r : RS) {
     if (r.span > 4096) {
       delete P;
@@ -461,16 +478,24 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
     }
     r.chunk = chunk;
     r.n_chunks = (int32_t)((r.key_hi + r.chunk - 1) / r.chunk);
-    // offsets one block of pass 2 touches: the rows' spread, its chunk and the look-back
-    const int32_t span64 = (r.span + 63) / 64 * 64;
-    sacc_n = std::max(sacc_n, r.span + chunk + span64 + 64);
+    if (r.slash_hi > r.slash_lo) max_span = std::max(max_span, r.span);
   }
+  for (auto& t : LT) {
+    t.key_hi = RS[t.rs[0]].key_hi;
+    t.n_chunks = RS[t.rs[0]].n_chunks;
+    if (t.rs[1] >= 0) {
+      t.key_hi = std::max(t.key_hi, RS[t.rs[1]].key_hi);
+      t.n_chunks = std::max(t.n_chunks, RS[t.rs[1]].n_chunks);
+    }
+  }
+  const int32_t lq_ring = lastq_ring_entries(max_span);
 
   // ---- layout
   lay.header = B.take(256);
   lay.classes = B.take((int64_t)sizeof(ClassStatic) * C.size());
   lay.heads = B.take((int64_t)sizeof(HeadStatic) * Hq);
   lay.rowsets = B.take((int64_t)sizeof(RowSet) * RS.size());
+  lay.lq_tiles = B.take((int64_t)sizeof(LqTile) * std::max<size_t>(LT.size(), 1));
   // jobs are sized below (after raw slots exist); reserve the maximum: 2 + 4 per row set
   const int64_t max_jobs = (int64_t)RS.size() * 3 + 1;
   lay.jobs = B.take((int64_t)sizeof(TopkJob) * max_jobs);
@@ -626,6 +651,7 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   std::memcpy(P->blob.data() + lay.classes, C.data(), sizeof(ClassStatic) * C.size());
   std::memcpy(P->blob.data() + lay.heads, HS.data(), sizeof(HeadStatic) * Hq);
   if (!RS.empty()) std::memcpy(P->blob.data() + lay.rowsets, RS.data(), sizeof(RowSet) * RS.size());
+  if (!LT.empty()) std::memcpy(P->blob.data() + lay.lq_tiles, LT.data(), sizeof(LqTile) * LT.size());
   if (!P->jobs.empty()) std::memcpy(P->blob.data() + lay.jobs, P->jobs.data(), sizeof(TopkJob) * P->jobs.size());
   std::memcpy(P->blob.data() + lay.items, P->items.data(), sizeof(WorkItem) * P->items.size());
   if (!P->bands.empty()) std::memcpy(P->blob.data() + lay.bands, P->bands.data(), sizeof(UnitBand) * P->bands.size());
@@ -668,7 +694,8 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   for (const auto& r : RS) mc = std::max(mc, r.n_chunks);
   dp.tb_words = tbw;
   dp.max_chunks = mc;
-  dp.sacc_n = sacc_n;
+  dp.n_lqtiles = (int32_t)LT.size();
+  dp.lq_ring = lq_ring;
   dp.class_kind = P->class_kind.data();
   *out = P;
   return MSA_OK;
@@ -922,6 +949,20 @@ msa_status msa_tile_stats(const msa_plan* P, const void* ws, int64_t tiles[2], v
   }
   tiles[0] = t;
   tiles[1] = n;
+  return MSA_OK;
+}
+
+msa_status msa_tile_stats_heads(const msa_plan* P, const void* ws, int64_t* tiles, void* stream) {
+  if (!P || !ws || !tiles) return MSA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  std::vector<int32_t> nt(P->items.size());
+  if (cudaMemcpyAsync(nt.data(), static_cast<const uint8_t*>(ws) + P->lay.item_ntiles, 4 * nt.size(),
+                      cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return MSA_ERR_CUDA;
+  for (int32_t h = 0; h < P->Hq; ++h) tiles[h] = 0;
+  for (size_t i = 0; i < nt.size(); ++i)
+    if (nt[i] > 0) tiles[P->classes[P->items[i].cls].head] += nt[i];
   return MSA_OK;
 }
 

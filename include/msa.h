@@ -220,6 +220,12 @@ msa_status msa_read_indices(const msa_plan* plan, const void* ws, int32_t head, 
  * Executed block FLOPs = 4 * 128 * 128 * 128 * tiles[0]. */
 msa_status msa_tile_stats(const msa_plan* plan, const void* ws, int64_t tiles[2], void* stream);
 
+/* Executed 128 x 128 tiles of each query head (host int64 [Hq]) under the tile lists of the last
+ * msa_estimate / msa_set_indices in `ws` (the FLOPs accounting of the MInference 1.0 and MMInference
+ * pages, per head: how much of the dense causal work each head's pattern executes).  Reads the
+ * per-item tile counts on `stream` and synchronises it. */
+msa_status msa_tile_stats_heads(const msa_plan* plan, const void* ws, int64_t* tiles, void* stream);
+
 /* Allowed (query, key) pairs of each query head under the masks of the last msa_estimate /
  * msa_set_indices in this workspace: causal in original positions and the head's pattern, each
  * pair once (MInference / MMInference: the token-level masks of the A-shape, vertical-slash,
