@@ -431,7 +431,13 @@ def measure_layer(args, name, rank, world, local_rank, steps, warmup, with_e2e, 
         assert plan_d.device_status(ws_d) == 0
         dense_ms = e0.elapsed_time(e1)
         dtiles, _ = plan_d.tile_stats(ws_d)
-        dense = {"attention_ms": dense_ms, "executed_flops": msa.executed_flops(dtiles),
+        # the pages' other sparsity statistic, on the dense layer's own rows: the share of the
+        # dense attention weights that 95 % of each row's softmax mass needs (stratified rows)
+        from dynamic_sparse_attention_head_b200.search import weight_share_stats
+        ws95 = weight_share_stats(p, q, k, rows_per_head=16, recall=0.95)
+        dense = {"weights_for_95pct_recall": {"mean_share": ws95["mean_share"], "per_kind": ws95["per_kind"],
+                                              "rows_per_head": ws95["rows_per_head"]},
+                 "attention_ms": dense_ms, "executed_flops": msa.executed_flops(dtiles),
                  "tflops": msa.executed_flops(dtiles) / (dense_ms * 1e-3) / 1e12,
                  "speedup_vs_dense_same_kernel": dense_ms / attn_ms,
                  "layer_speedup_vs_dense_attention": dense_ms / ms_step}

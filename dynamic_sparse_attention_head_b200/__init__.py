@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 KINDS = {"dense": 0, "ashape": 1, "vslash": 2, "block": 3, "grid": 4, "qbound": 5, "bound2d": 6}
 KIND_NAMES = {v: k for k, v in KINDS.items()}
 MAX_STRIDES = 8
+HEAD_PER_SEGMENT = 1  # msa_head_cfg.flags: Q-boundary index per modality segment
 STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "alignment", 4: "workspace", 5: "unsupported",
           6: "cuda", 7: "device timeout", 8: "device bounds", 9: "state"}
 
@@ -28,7 +29,7 @@ _I32, _I64, _F32, _F64, _P = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, cty
 class HeadCfg(ctypes.Structure):
     _fields_ = [("kind", _I32), ("sink", _I32), ("local", _I32), ("k_v", _I32), ("k_s", _I32),
                 ("topk_blocks", _I32), ("block_budget", _F64), ("n_strides", _I32), ("strides", _I32 * MAX_STRIDES),
-                ("n_phases", _I32), ("_pad", _I32), ("grid_budget", _F64)]
+                ("n_phases", _I32), ("flags", _I32), ("grid_budget", _F64)]
 
 
 class Segment(ctypes.Structure):
@@ -47,7 +48,8 @@ class Strides(ctypes.Structure):
 
 class HeadIndices(ctypes.Structure):
     _fields_ = [("stride", _I32), ("n_phases", _I32), ("phases", _P), ("n_v", (_I32 * 2) * 2),
-                ("v", (_P * 2) * 2), ("n_s", _I32 * 2), ("s", _P * 2), ("blk_ptr", _P), ("blk_idx", _P)]
+                ("v", (_P * 2) * 2), ("n_s", _I32 * 2), ("s", _P * 2), ("blk_ptr", _P), ("blk_idx", _P),
+                ("n_seg", _I32), ("seg_nv", _P), ("seg_v", _P), ("seg_ns", _P), ("seg_s", _P)]
 
 
 class MsaError(RuntimeError):
@@ -83,6 +85,8 @@ def _load():
         "msa_status_string": ([_I32], ctypes.c_char_p),
         "msa_kernel_launches": ([], ctypes.c_uint64),
         "msa_vslash_estimate_static": ([_P, _P, _I64, _I64, _I64, _F32, _I32, _I32, _P, _P, _P, _P], _I32),
+        "msa_weight_share": ([_P, _P, _I64, _I32, _I32, ctypes.POINTER(Strides), _F32, _P, _P, _I32, ctypes.c_double,
+                              _P, _P], _I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -96,7 +100,7 @@ EXPORTS = ("msa_plan_create", "msa_plan_destroy", "msa_workspace_bytes", "msa_wo
            "msa_sparse_prefill_indexed", "msa_estimate", "msa_set_indices",
            "msa_permute", "msa_sparse_prefill", "msa_unpermute", "msa_read_indices", "msa_read_tiles",
            "msa_tile_stats", "msa_tile_stats_heads", "msa_attention_units", "msa_mask_pairs", "msa_selftest_timeout", "msa_device_status", "msa_status_string",
-           "msa_kernel_launches", "msa_vslash_estimate_static")
+           "msa_kernel_launches", "msa_vslash_estimate_static", "msa_weight_share")
 
 
 def kernel_launches() -> int:
@@ -125,6 +129,7 @@ def _head_cfg(h) -> HeadCfg:
     for i, s in enumerate(st[:MAX_STRIDES]):
         c.strides[i] = int(s)
     c.n_phases, c.grid_budget = int(h.n_phases), float(h.grid_budget)
+    c.flags = HEAD_PER_SEGMENT if getattr(h, "per_segment", False) else 0
     return c
 
 
@@ -200,6 +205,17 @@ class Plan:
             if kind == "vslash":
                 hi.v[0][0], hi.n_v[0][0] = ptr(x["V"])
                 hi.s[0], hi.n_s[0] = ptr(x["S"])
+            elif kind == "qbound" and getattr(self.problem.heads[h], "per_segment", False):
+                nseg = len(self.problem.segments)
+                vp, sp = (_P * nseg)(), (_P * nseg)()
+                nv, ns = np.zeros(nseg, np.int32), np.zeros(nseg, np.int32)
+                for k in range(nseg):
+                    vp[k], nv[k] = ptr(x["V"][k])
+                    sp[k], ns[k] = ptr(x["S"][k])
+                keep += [vp, sp, nv, ns]
+                hi.n_seg = nseg
+                hi.seg_nv, hi.seg_ns = nv.ctypes.data, ns.ctypes.data
+                hi.seg_v, hi.seg_s = ctypes.cast(vp, _P), ctypes.cast(sp, _P)
             elif kind == "qbound":
                 for a, v in x["V"].items():
                     hi.v[a][0], hi.n_v[a][0] = ptr(v)
@@ -297,19 +313,34 @@ class Plan:
             s[a] = take(n)
         nb = r[i]
         i += 1
+        T = None
+        if kind == "block":
+            ptrs = take(nb + 1)
+            flat = take(int(ptrs[-1]))
+            T = [flat[ptrs[b]:ptrs[b + 1]] for b in range(nb)]
+        nseg = r[i]
+        i += 1
+        segv, segs = {}, {}
+        for k in range(nseg):  # per-segment Q-boundary: each segment's vertical and slash lines
+            n = r[i]
+            i += 1
+            segv[k] = take(n)
+            n = r[i]
+            i += 1
+            segs[k] = take(n)
         out = {"kind": kind}
         if kind == "grid":
             out.update(stride=stride, phases=phases)
         elif kind == "vslash":
             out.update(V=v[(0, 0)], S=s[0])
+        elif kind == "qbound" and nseg > 0:
+            out.update(per_segment=True, V=segv, S=segs)
         elif kind == "qbound":
             out.update(V={a: v[(a, 0)] for a in (0, 1)}, S=s)
         elif kind == "bound2d":
             out.update(V=v, S=s)
         elif kind == "block":
-            ptrs = take(nb + 1)
-            flat = take(int(ptrs[-1]))
-            out["T"] = [flat[ptrs[b]:ptrs[b + 1]] for b in range(nb)]
+            out["T"] = T
         return out
 
     def read_tiles(self, head: int, ws, stream=None) -> List[Dict]:
@@ -383,6 +414,22 @@ def vslash_estimate_static(Qh, Kh, scale: float, k_v: int, k_s: int, v_out, s_ou
            _lib.msa_vslash_estimate_static(Qh.data_ptr(), Kh.data_ptr(), Qh.shape[0], Qh.stride(0), Kh.stride(0),
                                            float(scale), int(k_v), int(k_s), v_out.data_ptr(), s_out.data_ptr(),
                                            counts_out.data_ptr(), _stream_ptr(stream)))
+
+
+def weight_share(Q, K, scale: float, heads, rows, recall: float = 0.95, stream=None):
+    """msa_weight_share: for each sample s, the fewest dense causal attention weights of query
+    row rows[s] of head heads[s] whose sum reaches `recall` of the row's softmax mass.
+    Q [Hq, L, 128], K [Hkv, L, 128]: bf16 CUDA tensors; heads, rows: int32 CUDA tensors [n].
+    Returns an int64 CUDA tensor [n] (the share of row i is count / (i + 1))."""
+    import torch
+    assert Q.dim() == 3 and K.dim() == 3 and Q.stride(2) == 1 and K.stride(2) == 1
+    n = int(rows.numel())
+    out = torch.empty(n, dtype=torch.int64, device=Q.device)
+    _check("msa_weight_share",
+           _lib.msa_weight_share(Q.data_ptr(), K.data_ptr(), Q.shape[1], Q.shape[0], K.shape[0],
+                                 ctypes.byref(_strides(Q, K)), float(scale), heads.data_ptr(), rows.data_ptr(), n,
+                                 float(recall), out.data_ptr(), _stream_ptr(stream)))
+    return out
 
 
 def executed_flops(tiles: int) -> int:

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmsa.so")
-SOURCES = ["plan.cu", "attn.cu", "index.cu", "estimate.cu", "lastq.cu", "permute.cu", "noalloc.cu", "selftest.cu"]
+SOURCES = ["plan.cu", "attn.cu", "index.cu", "estimate.cu", "lastq.cu", "permute.cu", "noalloc.cu", "selftest.cu", "recall.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
          "--expt-relaxed-constexpr"]

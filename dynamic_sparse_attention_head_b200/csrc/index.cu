@@ -92,9 +92,12 @@ __global__ void mat_lists_kernel(DevPlan dp) {
     ebits[w] = 0u;
   }
   __syncthreads();
+  // a class with its own lists (one class per segment) or the head's lists of modality a
+  const bool own = (cs.flags & CF_SEGIDX) != 0;
+  const int32_t* ccnt = own ? at<const int32_t>(dp, cs.segcnt_off) : nullptr;
   // slash lines
-  const int32_t ns = hs.raws_cap[a] > 0 ? counts[4 + a] : 0;
-  const int32_t* sl = at<const int32_t>(dp, hs.raws_off[a]);
+  const int32_t ns = own ? ccnt[1] : (hs.raws_cap[a] > 0 ? counts[4 + a] : 0);
+  const int32_t* sl = at<const int32_t>(dp, own ? cs.segs_off : hs.raws_off[a]);
   for (int i = threadIdx.x; i < ns; i += blockDim.x) {
     const int32_t o = sl[i];
     if (o < 0 || o >= dp.L) { flag_bounds(dp); continue; }
@@ -102,8 +105,8 @@ __global__ void mat_lists_kernel(DevPlan dp) {
   }
   // gathered keys: VSLASH [0][0]; QBOUND [a][0]; BOUND2D merge of [a][0] and [a][1]
   int32_t* xp = at<int32_t>(dp, cs.x_pos_off);
-  const int32_t* ra = at<const int32_t>(dp, hs.rawv_off[a][0]);
-  const int32_t na = hs.rawv_cap[a][0] > 0 ? counts[a * 2] : 0;
+  const int32_t* ra = at<const int32_t>(dp, own ? cs.segv_off : hs.rawv_off[a][0]);
+  const int32_t na = own ? ccnt[0] : (hs.rawv_cap[a][0] > 0 ? counts[a * 2] : 0);
   const int32_t* rb = at<const int32_t>(dp, hs.rawv_off[a][1]);
   const int32_t nb_ = (cs.kind == MSA_BOUND2D && hs.rawv_cap[a][1] > 0) ? counts[a * 2 + 1] : 0;
   const int32_t nx = na + nb_;

@@ -76,20 +76,23 @@ struct __align__(1024) LqtSmem {
   int abort;
 };
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+// tcgen05.wait::ld with the loaded registers as operands, so that no use of them can be
+// scheduled before the wait
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,"
-      "%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
-        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
-        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-      : "r"(taddr));
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+__device__ __forceinline__ float lq_fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // Barrier of the 64 softmax threads of one row set (named barriers 1 and 2).
@@ -288,13 +291,18 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
       // the warp decides together (the loads below are warp-collective)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[buf], (b >> 1) & 1, abort))) return false;
       tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld64(s_lane + (uint32_t)(buf * LQ_KB), sv);
-      tmem_wait_ld();
+      // the row in two 32-column loads: the first half is scaled while the second is in flight
+      uint32_t sa[32], sb[32];
+      tmem_ld32(s_lane + (uint32_t)(buf * LQ_KB), sa);
+      tmem_wait_ld_regs(sa);
+      tmem_ld32(s_lane + (uint32_t)(buf * LQ_KB + 32), sb);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sa[c]) * sl2;
+      tmem_wait_ld_regs(sb);
       tc_fence_before();
       mbar_arrive(&sm.s_free[buf]);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sv[c]) * sl2;
+      for (int c = 0; c < 32; ++c) x[32 + c] = __uint_as_float(sb[c]) * sl2;
       if (__any_sync(0xFFFFFFFFu, bmax > pr)) {  // some key of the block is after some row of the warp
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -310,20 +318,25 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
       for (int b = 0; b < nblk; ++b) {
         float x[64];
         if (!load_logits(b, x)) break;
-        float bm = -INFINITY;
+        // block max in eight independent chains of three-input maxima, then the sum of the
+        // exponentials in four chains (short dependency chains: the loop is latency-bound)
+        float m8[8];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) bm = fmaxf(bm, x[c]);
+        for (int q = 0; q < 8; ++q) m8[q] = x[q];
+#pragma unroll
+        for (int c = 8; c < 64; c += 16) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) m8[q] = lq_fmax3(m8[q], x[c + q], x[c + 8 + q]);
+        }
+        const float bm = fmaxf(lq_fmax3(m8[0], m8[1], m8[2]), lq_fmax3(m8[3], lq_fmax3(m8[4], m8[5], m8[6]), m8[7]));
         const float nm = fmaxf(mrun, bm);
         if (nm == -INFINITY) continue;
         z = (mrun == -INFINITY) ? 0.f : z * ex2(mrun - nm);
         mrun = nm;
-        float a0 = 0.f, a1 = 0.f;
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          a0 += ex2(x[c] - mrun);
-          a1 += ex2(x[c + 1] - mrun);
-        }
-        z += a0 + a1;
+        for (int c = 0; c < 64; ++c) a[c & 3] += ex2(x[c] - mrun);
+        z += (a[0] + a[1]) + (a[2] + a[3]);
       }
       if (rs != nullptr && chunk < rs->n_chunks) {
         float* mz = at<float>(dp, rs->mz_off) + (int64_t)chunk * LASTQ * 2;
@@ -357,6 +370,8 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
       float* sout = slash ? at<float>(dp, rs->s_off) : nullptr;
       const int32_t slo = slash ? rs->slash_lo : 0, shi = slash ? rs->slash_hi : 0;
       const int n_rows = rs != nullptr ? rs->n_rows : 0;
+      const int64_t rc0 = rs != nullptr ? rs->rcs[0] : 0;
+      const int64_t own_end = ck.own0 + ra.chunk;  // offsets owned: last-row key in [own0, own_end)
       set_sync(set);  // ring and row coordinates in place
 
       for (int b = 0; b < nblk; ++b) {
@@ -368,30 +383,36 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
           for (int c = 0; c < 64; ++c) P[rr * P_PITCH + c] = live ? ex2(x[c] - Mr) * Ir : 0.f;
         }
         if (set_any(set, !got)) break;  // every thread of the set leaves together
-        // vertical sums of the keys the chunk owns: column rr, rows in order
+        // vertical sums of the keys the chunk owns: column rr, rows in a fixed order (four
+        // interleaved partial sums, so that the loads overlap)
         {
           const int64_t j = j0 + rr;
           if (vout != nullptr && j >= own0 && j < own1) {
-            float a = 0.f;
-#pragma unroll 8
-            for (int r = 0; r < 64; ++r) a += P[r * P_PITCH + rr];
-            vout[j] = a;
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 16
+            for (int r = 0; r < 64; ++r) a[r & 3] += P[r * P_PITCH + rr];
+            vout[j] = (a[0] + a[1]) + (a[2] + a[3]);
           }
         }
         if (slash) {
           const bool inside = j0 >= slo && j0 + LQ_KB <= shi;
           if (contig) {
             // consecutive row coordinates: offset rc0 - j0 + d collects diagonal d = r - c of the
-            // block; this thread sums diagonals rr - 63 (rows 0..rr) and rr + 1 (rows rr+1..63)
-            float d1 = 0.f, d2 = 0.f;
+            // block; this thread sums diagonals rr - 63 (rows 0..rr) and rr + 1 (rows rr+1..63):
+            // row i contributes column (i + 63 - rr) mod 64 to one of the two (four interleaved
+            // partial sums each, combined in a fixed order)
+            float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 16
             for (int i = 0; i < 64; ++i) {
-              const int c = i <= rr ? i + 63 - rr : i - rr - 1;
+              const int c = (i + 63 - rr) & 63;
               float v = P[i * P_PITCH + c];
               if (!inside && (j0 + c < slo || j0 + c >= shi)) v = 0.f;
-              if (i <= rr) d1 += v;
-              else d2 += v;
+              const bool lo = i <= rr;
+              a1[i & 3] += lo ? v : 0.f;
+              a2[i & 3] += lo ? 0.f : v;
             }
-            const int64_t base = (int64_t)rs->rcs[0] - j0;
+            const float d1 = (a1[0] + a1[1]) + (a1[2] + a1[3]), d2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
+            const int64_t base = rc0 - j0;
             ring[(base + rr - 63) & (R - 1)] += d1;
             if (rr < 63) ring[(base + rr + 1) & (R - 1)] += d2;
           } else {
@@ -414,7 +435,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
           // offsets whose last-row key is j0 + rr are complete: written if the chunk owns them
           const int64_t o = (int64_t)max_rc - (j0 + rr);
           float& e = ring[o & (R - 1)];
-          if (j0 + rr >= own0 && j0 + rr < ck.own0 + ra.chunk && o >= 0 && o < dp.L) sout[o] = e;
+          if (j0 + rr >= own0 && j0 + rr < own_end && o >= 0 && o < dp.L) sout[o] = e;
           e = 0.f;
         }
       }
@@ -488,15 +509,16 @@ size_t lastq_smem_bytes(int pass, int ring) {
 }
 
 int32_t lastq_pick_chunk(const int32_t* tile_key_hi, int n_tiles) {
-  // the largest power of two from 8192 down to 256 keys that still gives four CTAs per SM, so
-  // that the look-back of pass 2 (the rows' span below each chunk) stays small against it
+  // the largest power of two from 8192 down to 256 keys that still gives eight CTAs per SM (four
+  // waves of the two resident CTAs, so that the last wave's tail is short), while the look-back
+  // of pass 2 (the rows' span below each chunk) stays small against the chunk
   auto ctas = [&](int32_t ch) {
     int64_t n = 0;
     for (int i = 0; i < n_tiles; ++i) n += (tile_key_hi[i] + ch - 1) / ch;
     return n;
   };
   int32_t chunk = 8192;
-  while (chunk > 256 && ctas(chunk) < 4LL * sm_count()) chunk /= 2;
+  while (chunk > 256 && ctas(chunk) < 8LL * sm_count()) chunk /= 2;
   return chunk;
 }
 

@@ -35,7 +35,8 @@ enum : int32_t {
   CF_X = 64,         // gathered key list present
   CF_DYNROWS = 128,  // row count decided on the device (grid heads)
   CF_SINK = 256,     // sink prefix
-  CF_BAND = 512      // local band
+  CF_BAND = 512,     // local band
+  CF_SEGIDX = 1024   // the class's vertical / slash lists are its own (one class per segment)
 };
 
 // Device error bits recorded in the workspace header.
@@ -55,7 +56,7 @@ struct ClassStatic {
   int32_t qrow0_static;    // first row in the head's permuted Q / O slice (static classes)
   int32_t item0, n_items;  // work items [item0, item0 + n_items)
   int32_t tile_cap;        // tile capacity per work item
-  int32_t _pad0;
+  int32_t seg;             // CF_SEGIDX: the segment whose queries the class holds, else -1
   int64_t rows_off;        // int32 [max_rows] original positions of the rows (CF_PERMUTED)
   int64_t x_pos_off;       // int32 [x_cap] positions of gathered keys, POS_PAD padded
   int64_t slash_list_off;  // int32 slash offsets (sorted) - raw list
@@ -65,6 +66,9 @@ struct ClassStatic {
   int64_t tile_base;       // first tile slot of item slot 0 (item slot s starts at tile_base + s * tile_cap)
   int32_t blk_wpr;         // words per block-bitmap row
   int32_t dyn;             // index into the ClassDyn array
+  // CF_SEGIDX: the class's raw lists (positions, offsets) and their counts (int32 [2]: n_v, n_s)
+  int64_t segv_off, segs_off, segcnt_off;
+  int32_t segv_cap, segs_cap;
 };
 
 // Written on the device every prefill.
@@ -114,6 +118,8 @@ struct RowSet {
   int64_t mz_off;            // fp32 [n_chunks][LASTQ][2] partial (max, sum) of pass 1
   int64_t stat_off;          // fp32 [LASTQ][2] row max and 1/sum
   int32_t n_chunks, chunk;   // key chunks of the sweep
+  int32_t cls;               // class whose own lists this row set's index fills (CF_SEGIDX), else -1
+  int32_t _pad;
 };
 
 // One tile of the last-query sweep: up to two row sets of one KV head and key source, stacked

@@ -155,6 +155,7 @@ extern "C" msa_status msa_vslash_estimate_static(const void* Q, const void* K, i
   r.stat_off = stat_off;
   r.chunk = chunk;
   r.n_chunks = n_chunks;
+  r.cls = -1;
   t.tile.rs[0] = 0;
   t.tile.rs[1] = -1;
   t.tile.kvh = 0;

@@ -99,6 +99,8 @@ msa_status validate(const msa_problem* p) {
     if (c.kind == MSA_VSLASH || c.kind == MSA_QBOUND || c.kind == MSA_BOUND2D)
       if (c.k_v < 1 || c.k_s < 1) return MSA_ERR_INVALID_ARG;
     if (c.kind == MSA_BLOCK && c.topk_blocks == 0 && !(c.block_budget > 0.0)) return MSA_ERR_INVALID_ARG;
+    if ((c.flags & ~MSA_HEAD_PER_SEGMENT) || ((c.flags & MSA_HEAD_PER_SEGMENT) && c.kind != MSA_QBOUND))
+      return MSA_ERR_INVALID_ARG;
     if (c.kind == MSA_GRID) {
       if (c.n_strides < 1 || c.n_strides > MSA_MAX_STRIDES) return MSA_ERR_INVALID_ARG;
       for (int i = 0; i < c.n_strides; ++i)
@@ -158,7 +160,16 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   const int32_t Hq = P->Hq, Hkv = P->Hkv, G = Hq / Hkv;
   const int64_t nb = L / BLK;
   const int64_t nwords = (L + 31) / 32;
-  const int32_t LP = (int32_t)(round_up(L, TILE) + 2 * TILE);
+  // rows of a head's permuted Q / O slice: classes start at multiples of 128 rows; a head with
+  // one class per segment needs the segments' lengths rounded up
+  int64_t lp = round_up(L, TILE) + 2 * TILE;
+  for (int32_t h = 0; h < prob->Hq; ++h)
+    if (prob->heads[h].flags & MSA_HEAD_PER_SEGMENT) {
+      int64_t r = 2 * TILE;
+      for (int i = 0; i < prob->n_segments; ++i) r += round_up(prob->segments[i].len, TILE);
+      lp = std::max(lp, r);
+    }
+  const int32_t LP = (int32_t)lp;
   P->mod.assign(L, 0);
   P->rank.assign(L, 0);
   for (const auto& s : P->segs)
@@ -203,6 +214,7 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
       c.max_rows = (int32_t)L;
       c.rows_static = (int32_t)L;
       c.qrow0_static = 0;
+      c.seg = -1;
       return c;
     };
     switch (cfg.kind) {
@@ -263,6 +275,26 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
         break;
       }
       case MSA_QBOUND:
+        if (cfg.flags & MSA_HEAD_PER_SEGMENT) {
+          // one class per segment: its queries (a contiguous run of its modality's positions)
+          // with their own vertical and slash lines
+          int32_t q0 = 0;
+          for (int k = 0; k < (int)P->segs.size(); ++k) {
+            const msa_segment& sg = P->segs[k];
+            ClassStatic c = base(CF_PERMUTED | CF_X | CF_SLASH | CF_EXCL | CF_SEGIDX);
+            c.modality = sg.modality;
+            c.seg = k;
+            c.max_rows = c.rows_static = (int32_t)sg.len;
+            c.qrow0_static = q0;
+            q0 += (int32_t)round_up(sg.len, TILE);
+            c.x_cap = (int32_t)round_up(std::min<int64_t>(cfg.k_v, L), TILE);
+            c.segv_cap = (int32_t)std::min<int64_t>(cfg.k_v, L);
+            c.segs_cap = (int32_t)std::min<int64_t>(cfg.k_s, L);
+            C.push_back(c);
+          }
+          break;
+        }
+        [[fallthrough]];
       case MSA_BOUND2D: {
         const bool two = cfg.kind == MSA_BOUND2D;
         for (int a = 0; a < 2; ++a) {
@@ -392,12 +424,21 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   std::vector<RowSet>& RS = P->rowsets;
   for (int32_t h = 0; h < Hq; ++h) {
     const msa_head_cfg& cfg = P->heads[h];
-    auto add = [&](int a_rows, int k_src, int32_t a_rank) -> int {
+    // a_rows: modality of the rows (-1: any); seg >= 0: rows of that segment only
+    auto add = [&](int a_rows, int k_src, int32_t a_rank, int seg = -1) -> int {
       RowSet r{};
       r.head = h;
       r.kvh = h / G;
       r.k_src = k_src;
-      std::vector<int32_t> rows = last_rows(*P, a_rows);
+      r.cls = -1;
+      std::vector<int32_t> rows;
+      if (seg >= 0) {
+        const msa_segment& sg = P->segs[seg];
+        for (int64_t t = std::max<int64_t>(sg.start, sg.start + sg.len - LASTQ); t < sg.start + sg.len; ++t)
+          rows.push_back((int32_t)t);
+      } else {
+        rows = last_rows(*P, a_rows);
+      }
       r.n_rows = (int32_t)rows.size();
       int32_t lo = INT32_MAX, hi = INT32_MIN;
       for (int i = 0; i < r.n_rows; ++i) {
@@ -424,6 +465,16 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
         break;
       }
       case MSA_QBOUND:
+        if (cfg.flags & MSA_HEAD_PER_SEGMENT) {
+          // the last 64 queries of every segment, feeding that segment's class
+          for (int c = HS[h].class0; c < HS[h].class0 + HS[h].n_classes; ++c) {
+            int i = add(C[c].modality, SRC_K, -1, C[c].seg);
+            RS[i].slash_lo = 0;
+            RS[i].slash_hi = (int32_t)L;
+            RS[i].cls = c;
+          }
+          break;
+        }
         for (int a = 0; a < 2; ++a) {
           if (P->n_mod[a] == 0) continue;
           int i = add(a, SRC_K, -1);
@@ -522,7 +573,8 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
     HeadStatic& H = HS[h];
     const msa_head_cfg& cfg = P->heads[h];
     H.counts_off = B.take(64);
-    if (cfg.kind == MSA_VSLASH || cfg.kind == MSA_QBOUND || cfg.kind == MSA_BOUND2D) {
+    const bool per_seg = (cfg.flags & MSA_HEAD_PER_SEGMENT) != 0;  // lists live in the classes
+    if ((cfg.kind == MSA_VSLASH || cfg.kind == MSA_QBOUND || cfg.kind == MSA_BOUND2D) && !per_seg) {
       for (int a = 0; a < 2; ++a) {
         if (P->n_mod[a] == 0 && cfg.kind != MSA_VSLASH) continue;
         if (cfg.kind == MSA_VSLASH && a > 0) continue;
@@ -563,12 +615,19 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   for (auto& c : C) {
     const HeadStatic& H = HS[c.head];
     if (c.flags & CF_DYNROWS) c.rows_off = B.take(4 * L);
+    else if (c.flags & CF_SEGIDX)  // the segment's positions: a run of its modality's list
+      c.rows_off = lay.mod_rows[c.modality] + 4 * (int64_t)P->rank[P->segs[c.seg].start];
     else if (c.flags & CF_PERMUTED) c.rows_off = lay.mod_rows[c.modality];
+    if (c.flags & CF_SEGIDX) {
+      c.segv_off = B.take(4 * (int64_t)std::max(c.segv_cap, 1));
+      c.segs_off = B.take(4 * (int64_t)std::max(c.segs_cap, 1));
+      c.segcnt_off = B.take(8);
+    }
     if (c.flags & CF_X) c.x_pos_off = B.take(4 * (int64_t)c.x_cap);
     if (c.flags & CF_SLASH) {
       c.slash_bits_off = B.take(4 * nwords);
       int a = (c.kind == MSA_VSLASH) ? 0 : c.modality;
-      c.slash_list_off = H.raws_off[a];
+      c.slash_list_off = (c.flags & CF_SEGIDX) ? c.segs_off : H.raws_off[a];
     }
     if (c.flags & CF_EXCL) c.excl_bits_off = B.take(4 * nwords);
     if (c.flags & CF_BLOCK) c.blk_bits_off = B.take(4 * nb * (int64_t)c.blk_wpr);
@@ -587,6 +646,26 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
     const int32_t maxrow = r.rows[r.n_rows - 1];
     int32_t maxrc = r.rcs[0];
     for (int i = 0; i < r.n_rows; ++i) maxrc = std::max(maxrc, r.rcs[i]);
+    if (r.cls >= 0) {  // a segment's own lists
+      const ClassStatic& c = C[r.cls];
+      TopkJob jv{};
+      jv.score_off = r.v_off;
+      jv.lo = 0;
+      jv.hi = maxrow + 1;
+      jv.k = c.segv_cap;
+      jv.out_off = c.segv_off;
+      jv.cnt_off = c.segcnt_off;
+      P->jobs.push_back(jv);
+      TopkJob js{};
+      js.score_off = r.s_off;
+      js.lo = 0;
+      js.hi = maxrc + 1;
+      js.k = c.segs_cap;
+      js.out_off = c.segs_off;
+      js.cnt_off = c.segcnt_off + 4;
+      P->jobs.push_back(js);
+      continue;
+    }
     if (cfg.kind == MSA_BOUND2D) {
       const int a = P->mod[r.rows[0]];
       for (int b = 0; b < 2; ++b) {
@@ -787,6 +866,22 @@ msa_status msa_set_indices(msa_plan* P, const msa_head_indices* heads, void* ws,
       }
       return true;
     };
+    if (P->heads[h].flags & MSA_HEAD_PER_SEGMENT) {  // one pair of lists per segment
+      if (x.n_seg != (int32_t)P->segs.size() || !x.seg_nv || !x.seg_v || !x.seg_ns || !x.seg_s)
+        return MSA_ERR_INVALID_ARG;
+      for (int c = H.class0; c < H.class0 + H.n_classes; ++c) {
+        const ClassStatic& cl = P->classes[c];
+        const int k = cl.seg;
+        const int32_t nv = x.seg_nv[k], ns = x.seg_ns[k];
+        if (nv > cl.segv_cap || !sorted_in(x.seg_v[k], nv, 0, L)) return MSA_ERR_INVALID_ARG;
+        if (ns > cl.segs_cap || !sorted_in(x.seg_s[k], ns, 0, L)) return MSA_ERR_INVALID_ARG;
+        puts.emplace_back(cl.segv_off, std::vector<int32_t>(x.seg_v[k], x.seg_v[k] + nv));
+        puts.emplace_back(cl.segs_off, std::vector<int32_t>(x.seg_s[k], x.seg_s[k] + ns));
+        puts.emplace_back(cl.segcnt_off, std::vector<int32_t>{nv, ns});
+      }
+      puts.emplace_back(H.counts_off, counts);
+      continue;
+    }
     switch (H.kind) {
       case MSA_VSLASH:
       case MSA_QBOUND:
@@ -1038,6 +1133,23 @@ msa_status msa_read_indices(const msa_plan* P, const void* ws, int32_t head, int
     for (int64_t b = 0; b < nb; ++b) rec.push_back(acc += cnt[b]);
     for (int64_t b = 0; b < nb; ++b)
       rec.insert(rec.end(), lists.begin() + b * H.blk_kmax, lists.begin() + b * H.blk_kmax + cnt[b]);
+  } else {
+    rec.push_back(0);
+  }
+  if (P->heads[head].flags & MSA_HEAD_PER_SEGMENT) {  // the lists of every segment, in order
+    rec.push_back(H.n_classes);
+    for (int c = H.class0; c < H.class0 + H.n_classes; ++c) {
+      const ClassStatic& cl = P->classes[c];
+      std::vector<int32_t> cnt = fetch(cl.segcnt_off, 2);
+      if (cudaStreamSynchronize(cs) != cudaSuccess) return MSA_ERR_CUDA;
+      const int32_t nv = std::min(std::max(cnt[0], 0), cl.segv_cap), ns = std::min(std::max(cnt[1], 0), cl.segs_cap);
+      std::vector<int32_t> v = fetch(cl.segv_off, nv), sl = fetch(cl.segs_off, ns);
+      if (cudaStreamSynchronize(cs) != cudaSuccess) return MSA_ERR_CUDA;
+      rec.push_back(nv);
+      rec.insert(rec.end(), v.begin(), v.end());
+      rec.push_back(ns);
+      rec.insert(rec.end(), sl.begin(), sl.end());
+    }
   } else {
     rec.push_back(0);
   }

@@ -71,7 +71,12 @@ enum { MSA_TEXT = 0, MSA_VIDEO = 1 };
  *  GRID    : video grid (MMInference Algorithm 1): stride s and phases P searched online from
  *            the last 64 video queries; queries and keys on the (s, P) lines attend / are attended
  *            densely, text queries attend densely, plus a local band of `local` (default 64).
- *  QBOUND  : Q-boundary (Algorithm 2): vertical-slash per query modality.
+ *  QBOUND  : Q-boundary (Algorithm 2): vertical-slash per query modality.  With the head flag
+ *            MSA_HEAD_PER_SEGMENT: vertical-slash per modality segment, each segment's lines
+ *            estimated from its own last 64 queries (all of them if shorter) and serving only
+ *            that segment's queries (the MMInference review page's "last 64 queries of each
+ *            modality segment", read literally; the default estimates once per modality, from
+ *            its last segment, and extrapolates across the others, "key machinery").
  *  BOUND2D : 2D-boundary (Algorithm 3): per (query modality, key modality) pair; intra-modality
  *            pairs are vertical-slash in within-modality ranks, cross pairs vertical only. */
 typedef enum {
@@ -97,9 +102,12 @@ typedef struct {
   int32_t n_strides;   /* GRID: candidate strides (1..MSA_MAX_STRIDES) */
   int32_t strides[MSA_MAX_STRIDES];
   int32_t n_phases;    /* GRID: phases kept (> 0), else max(1, floor(grid_budget * s / 2)) */
-  int32_t _pad;
+  int32_t flags;       /* MSA_HEAD_* options (0: none) */
   double grid_budget;
 } msa_head_cfg;
+
+/* msa_head_cfg.flags: QBOUND only, one index per modality segment (see MSA_QBOUND) */
+#define MSA_HEAD_PER_SEGMENT 1
 
 typedef struct {
   int64_t start, len; /* token range [start, start + len) */
@@ -162,6 +170,13 @@ typedef struct {
   const int32_t* s[2];
   const int32_t* blk_ptr;  /* BLOCK: CSR over query blocks, blk_ptr[L/64 + 1] */
   const int32_t* blk_idx;  /* BLOCK: selected key blocks (each row ascending, c <= b) */
+  /* QBOUND with MSA_HEAD_PER_SEGMENT: lines of each segment k (n_seg = the problem's segment
+   * count): vertical positions seg_v[k][0 .. seg_nv[k]) and slash offsets seg_s[k][0 .. seg_ns[k]) */
+  int32_t n_seg;
+  const int32_t* seg_nv;
+  const int32_t* const* seg_v;
+  const int32_t* seg_ns;
+  const int32_t* const* seg_s;
 } msa_head_indices;
 
 msa_status msa_set_indices(msa_plan* plan, const msa_head_indices* heads, void* ws, size_t ws_bytes,
@@ -210,6 +225,8 @@ msa_status msa_sparse_prefill_indexed(msa_plan* plan, const void* Q, const void*
  *   for a in {0,1}, b in {0,1}: n_v[a][b], v[a][b][...],
  *   for a in {0,1}: n_s[a], s[a][...],
  *   nb, blk_ptr[nb + 1], blk_idx[blk_ptr[nb]]          (nb = 0 unless BLOCK)
+ *   n_seg, then per segment k: n_v, v[...], n_s, s[...]  (n_seg = 0 unless QBOUND with
+ *                                                         MSA_HEAD_PER_SEGMENT)
  * `*len` is the capacity of `out` in int32 on entry and the record length on return
  * (MSA_ERR_INVALID_ARG with the needed length if too small). */
 msa_status msa_read_indices(const msa_plan* plan, const void* ws, int32_t head, int32_t* out, int64_t* len,
@@ -275,6 +292,22 @@ msa_status msa_device_status(const msa_plan* plan, void* ws, void* stream);
 msa_status msa_selftest_timeout(const msa_plan* plan, void* ws, uint32_t limit_us, void* stream);
 
 const char* msa_status_string(msa_status status);
+
+/* ---- attention analysis ----
+ *
+ * Share of the dense attention weights needed for a given recall (MMInference summary page,
+ * attention analysis: in video-language models 95 % of the attention mass lies in 1.79 % of the
+ * weights, against 5.78 % in language models).  For sample s, query row i = rows[s] of query
+ * head h = heads[s]: the dense causal weights w_j = softmax_j(q_i . k_j * scale), j <= i, taken
+ * in descending order; counts[s] = the fewest of them whose sum reaches recall * sum_j w_j
+ * (the share is counts[s] / (i + 1)).  Q [Hq][L][128] and K [Hkv][L][128] bf16 on the device
+ * with the q_* and k_* element strides of `strides` (multiples of 8; pointers 16-byte
+ * aligned); query head h reads KV head h / (Hq / Hkv).  heads, rows: device int32 [n]; counts:
+ * device int64 [n], -1 for a sample whose head or row is out of range.  recall in (0, 1].
+ * Logits in fp32, weights and sums in fp64.  Asynchronous on `stream`; allocates nothing. */
+msa_status msa_weight_share(const void* Q, const void* K, int64_t L, int32_t Hq, int32_t Hkv,
+                            const msa_strides* strides, float scale, const int32_t* heads, const int32_t* rows,
+                            int32_t n, double recall, int64_t* counts, void* stream);
 
 /* ---- allocation-free variant ----
  *

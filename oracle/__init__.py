@@ -35,6 +35,7 @@ LAST_Q = 64
 BLOCK = 64
 GRID_BAND = 64
 KIND_ID = {"dense": 0, "ashape": 1, "vslash": 2, "block": 3, "grid": 4, "qbound": 5, "bound2d": 6}
+K_QSEG = 7  # Q-boundary estimated per modality segment
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -50,7 +51,7 @@ def build(force: bool = False) -> str:
 class _Mask(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("_pad", ctypes.c_int32), ("sink", _I64), ("local", _I64),
                 ("vcol", _P * 4), ("slash", _P * 2), ("gmark", _P), ("modality", _P), ("rank", _P),
-                ("blocksel", _P), ("nb", _I64)]
+                ("blocksel", _P), ("nb", _I64), ("segid", _P), ("vseg", _P), ("sseg", _P)]
 
 
 def _load():
@@ -188,6 +189,21 @@ def estimate_head(p: Problem, h: int, Q: np.ndarray, K: np.ndarray) -> Dict:
     if head.kind == "grid":
         return _estimate_grid(p, head, Qh, Kh, mod, out)
 
+    if head.kind == "qbound" and head.per_segment:
+        # MMInference review page, "core discovery" (the last 64 queries of each modality
+        # segment), read literally: every segment k gets its own vertical-slash index from its
+        # own last 64 queries (all of them if it is shorter), over all causal keys, and that
+        # index serves the queries of segment k only.
+        out.update(per_segment=True, V={}, S={}, v={}, s={})
+        for k, (st, n, _) in enumerate(p.segments):
+            rows = last_rows(np.arange(st, st + n))
+            v, s = lastq_sums(Qh, Kh, p.scale, rows)
+            cand = (np.arange(L) <= rows.max()).astype(np.uint8)
+            out["V"][k] = topk(v, head.k_v, cand)
+            out["S"][k] = topk(s, head.k_s, cand)
+            out["v"][k], out["s"][k] = v, s
+        return out
+
     if head.kind == "qbound":
         # MMInference Algorithm 2 (Q-boundary): the query axis is split at modality
         # boundaries; each query modality gets its own vertical-slash index from the
@@ -321,6 +337,19 @@ class MaskArrays:
         if k == "vslash":
             m.vcol[0] = marks(idx["V"])
             m.slash[0] = marks(idx["S"])
+        elif k == "qbound" and head.per_segment:
+            m.kind = K_QSEG
+            segid = np.zeros(L, np.int32)
+            for kk, (st, n, _) in enumerate(p.segments):
+                segid[st:st + n] = kk
+            self.keep.append(segid)
+            m.segid = segid.ctypes.data
+            nseg = len(p.segments)
+            vptr = (_P * nseg)(*[marks(idx["V"][kk]) for kk in range(nseg)])
+            sptr = (_P * nseg)(*[marks(idx["S"][kk]) for kk in range(nseg)])
+            self.keep += [vptr, sptr]
+            m.vseg = ctypes.cast(vptr, _P)
+            m.sseg = ctypes.cast(sptr, _P)
         elif k == "qbound":
             for a, ix in idx["V"].items():
                 m.vcol[a * 2] = marks(ix)
@@ -401,6 +430,7 @@ def permutation(p: Problem, h: int, idx: Dict):
     Readings (the pages state the goal, contiguous selected entries, not an ordering):
       grid (Algorithm 1): queries and keys on the selected grid lines first, then the others;
       Q-boundary (Algorithm 2): queries grouped by modality (text, then video), keys unchanged;
+        estimated per segment, queries grouped by segment (the original order), keys unchanged;
       2D-boundary (Algorithm 3): queries and keys grouped by modality;
       vertical-slash: keys on the vertical lines first (the lines gathered), queries unchanged;
       other kinds: identity.
@@ -412,6 +442,8 @@ def permutation(p: Problem, h: int, idx: Dict):
     if kind == "grid":
         g = grid_marks(p, idx["stride"], idx["phases"]).astype(bool)
         return _front(g), _front(g)
+    if kind == "qbound" and p.heads[h].per_segment:
+        return ident, ident
     if kind == "qbound":
         return _front(mod == TEXT), ident
     if kind == "bound2d":
@@ -446,3 +478,23 @@ def attention_permuted(p: Problem, h: int, Q, K, V, idx: Dict, qperm, kperm):
     O[qperm] = Op
     lse[qperm] = lp
     return O, lse
+
+
+# --------------------------------------------------------------------------------------
+# attention analysis (MMInference summary page, attention-sparsity analysis)
+# --------------------------------------------------------------------------------------
+def weight_share(Q, K, scale: float, head: int, row: int, group: int, recall: float = 0.95):
+    """The fewest dense causal attention weights of query `row` of `head` whose sum reaches
+    `recall` of the row's softmax mass (the pages' statistic: the share of the weights that 95 %
+    recall needs).  Logits as everywhere in the oracle: fp64 dot products rounded to fp32, times
+    the fp32 scale; weights exp(x - max), the descending sort and the running sum in fp64.
+    Returns (count, running sum of the sorted weights divided by their total)."""
+    from workload import bf16_to_f32
+    q = bf16_to_f32(np.asarray(Q[head][row])).astype(np.float64)
+    k = bf16_to_f32(np.asarray(K[head // group][: row + 1])).astype(np.float64)
+    x = (k @ q).astype(np.float32) * np.float32(scale)
+    w = np.exp(x.astype(np.float64) - float(x.max()))
+    w = np.sort(w)[::-1]
+    cum = np.cumsum(w) / w.sum()
+    count = int(np.searchsorted(cum, recall, side="left")) + 1
+    return min(count, row + 1), cum

@@ -169,7 +169,7 @@ void orc_block_topk(const double* Qbar, const double* Kbar, int64_t nb, int d, f
 /* ---------------------------------------------------------------------------------- */
 /* token-level masks                                                                   */
 /* ---------------------------------------------------------------------------------- */
-enum { K_DENSE = 0, K_ASHAPE = 1, K_VSLASH = 2, K_BLOCK = 3, K_GRID = 4, K_QBOUND = 5, K_BOUND2D = 6 };
+enum { K_DENSE = 0, K_ASHAPE = 1, K_VSLASH = 2, K_BLOCK = 3, K_GRID = 4, K_QBOUND = 5, K_BOUND2D = 6, K_QSEG = 7 };
 
 typedef struct {
   int32_t kind;
@@ -187,6 +187,11 @@ typedef struct {
   const int64_t* rank;     /* rank of a token among the tokens of its modality */
   const uint8_t* blocksel; /* block-sparse: [nb][nb] selected (query block, key block) */
   int64_t nb;
+  /* Q-boundary estimated per segment: segid[t] = segment of token t; vseg[k] / sseg[k] mark the
+     vertical keys / slash offsets estimated for the queries of segment k */
+  const int32_t* segid;
+  const uint8_t* const* vseg;
+  const uint8_t* const* sseg;
 } orc_mask;
 
 /*
@@ -196,7 +201,9 @@ typedef struct {
  *  Block-sparse (MInference 1.0): the 64-token (query block, key block) pair was selected.
  *  Grid (MMInference Algorithm 1, "key machinery"): video queries and keys on the
  *    selected horizontal/vertical grid lines, text queries, plus a local band.
- *  Q-boundary (MMInference Algorithm 2): vertical-slash per query modality.
+ *  Q-boundary (MMInference Algorithm 2): vertical-slash per query modality; estimated per
+ *    modality segment, vertical-slash per query segment (the queries of segment k use the
+ *    lines estimated from segment k's last 64 queries).
  *  2D-boundary (MMInference Algorithm 3): per (query modality, key modality) pair;
  *    intra-modality pairs are vertical-slash in within-modality (compacted)
  *    coordinates, so slash lines continue across text-interrupted video;
@@ -223,6 +230,10 @@ static inline int allowed(const orc_mask* m, int64_t i, int64_t j) {
       int a = m->modality[i], b = m->modality[j];
       if (a == b) return m->vcol[a * 2 + a][j] || m->slash[a][m->rank[i] - m->rank[j]];
       return m->vcol[a * 2 + b][j] != 0;
+    }
+    case K_QSEG: {
+      const int32_t k = m->segid[i];
+      return m->vseg[k][j] || m->sseg[k][i - j];
     }
   }
   return 0;

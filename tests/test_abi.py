@@ -148,3 +148,41 @@ def test_workspace_size_and_state_checks_come_before_any_device_access():
     # the self-test's limit is bounded to (0, 1 s]
     assert _lib.msa_selftest_timeout(plan._h, ws, 0, None) == 1
     assert _lib.msa_selftest_timeout(plan._h, ws, 2000000, None) == 1
+
+
+def test_per_segment_flag_validation_and_slice_rows():
+    """The per-segment option is a Q-boundary flag only; a head with one class per segment gets a
+    permuted Q/O slice long enough for every segment rounded up to 128 rows."""
+    import dataclasses
+    import dynamic_sparse_attention_head_b200 as msa
+    from workload import TEXT, VIDEO, Head, Problem
+    segs = [(0, 64, TEXT), (64, 64, VIDEO)] * 8  # 16 segments of 64 tokens: 8K rows once rounded up
+    segs = [(i * 64, 64, m) for i, (_, _, m) in enumerate(segs)]
+    p = Problem(L=1024, Hq=1, Hkv=1, segments=segs, heads=[Head("qbound", k_v=8, k_s=8)])
+    base = msa.Plan(p).workspace_bytes
+    q = dataclasses.replace(p, heads=[Head("qbound", k_v=8, k_s=8, per_segment=True)])
+    assert msa.Plan(q).workspace_bytes > base
+    bad = msa.HeadCfg()
+    bad.kind, bad.k_v, bad.k_s, bad.flags = msa.KINDS["vslash"], 8, 8, msa.HEAD_PER_SEGMENT
+    import pytest
+    with pytest.raises(msa.MsaError) as e:
+        _plan_with_cfg(p, bad)
+    assert e.value.code == 1
+    ok = msa.HeadCfg()
+    ok.kind, ok.k_v, ok.k_s, ok.flags = msa.KINDS["qbound"], 8, 8, msa.HEAD_PER_SEGMENT
+    _plan_with_cfg(p, ok)
+
+
+def _plan_with_cfg(p, cfg):
+    """msa_plan_create on problem p with its heads replaced by the raw configuration cfg."""
+    import ctypes
+    import dynamic_sparse_attention_head_b200 as msa
+    segs = (msa.Segment * len(p.segments))()
+    for i, (s, n, m) in enumerate(p.segments):
+        segs[i].start, segs[i].len, segs[i].modality = s, n, m
+    heads = (msa.HeadCfg * p.Hq)(*([cfg] * p.Hq))
+    pc = msa.ProblemC(L=p.L, Hq=p.Hq, Hkv=p.Hkv, d=p.d, scale=p.scale, n_segments=len(p.segments),
+                      segments=ctypes.cast(segs, ctypes.c_void_p), heads=ctypes.cast(heads, ctypes.c_void_p))
+    h = ctypes.c_void_p()
+    msa._check("msa_plan_create", msa._lib.msa_plan_create(ctypes.byref(pc), ctypes.byref(h)))
+    msa._lib.msa_plan_destroy(h)

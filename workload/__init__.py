@@ -67,9 +67,13 @@ class Head:
     strides: Tuple[int, ...] = ()
     n_phases: int = 0
     grid_budget: float = 0.0
+    # Q-boundary heads: estimate from the last 64 queries of each modality segment and apply each
+    # index to its own segment (instead of one index per modality)
+    per_segment: bool = False
 
     def __post_init__(self):
         assert self.kind in KINDS, self.kind
+        assert not self.per_segment or self.kind == "qbound", "per-segment estimation is a Q-boundary option"
 
 
 @dataclass
