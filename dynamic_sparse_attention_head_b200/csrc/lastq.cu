@@ -49,7 +49,8 @@ __host__ __device__ __forceinline__ T* at(const DevPlan& dp, int64_t off) {
 
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int LQ_KB = 64;                       // keys per block (MMA N)
-constexpr int LQ_THREADS = 192;                 // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int LQ_THREADS = 320;                 // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int LQ_SOFTMAX = 256;                 // softmax threads: two per query row
 constexpr uint32_t Q_ATOM = 128 * 128;          // [128 rows][64 cols] bf16, 128-byte swizzled
 constexpr uint32_t K_ATOM = LQ_KB * 128;        // [64 rows][64 cols]
 constexpr uint32_t K_STAGE = 2 * K_ATOM;        // one 64-key block, all 128 columns
@@ -95,10 +96,10 @@ __device__ __forceinline__ float lq_fmax3(float a, float b, float c) {
   return r;
 }
 
-// Barrier of the 64 softmax threads of one row set (named barriers 1 and 2).
+// Barrier of the 128 softmax threads of one row set (named barriers 1 and 2).
 __device__ __forceinline__ void set_sync(int set) {
-  if (set == 0) asm volatile("bar.sync 1, 64;" ::: "memory");
-  else asm volatile("bar.sync 2, 64;" ::: "memory");
+  if (set == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+  else asm volatile("bar.sync 2, 128;" ::: "memory");
 }
 
 // The tile's key range processed by chunk `chunk`: keys [c0, c1), of which the chunk owns
@@ -135,14 +136,14 @@ struct LqtSmem2 {
   int32_t rcs[2][64];
 };
 
-// bar.red.or over the 64 threads of one row set: true if any of them passes true.
+// bar.red.or over the 128 threads of one row set: true if any of them passes true.
 template <int ID>
 __device__ __forceinline__ bool bar_any(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, 64, p;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)v), "n"(ID)
@@ -183,9 +184,9 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 128);
+      mbar_init(&sm.s_free[b], LQ_SOFTMAX);
     }
-    mbar_init(&sm.q_ready, 128);
+    mbar_init(&sm.q_ready, LQ_SOFTMAX);
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
@@ -241,13 +242,17 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
-    const int qd = warp & 3;  // a warp reaches TMEM lanes 32 (warp % 4) .. + 31 only
+    // eight warps, two per row: warp w reaches TMEM lanes 32 (w % 4) .. + 31 only, so warps
+    // 2-5 take columns 0-31 of their 32 rows and warps 6-9 columns 32-63 of the same rows
+    const int qd = warp & 3;
+    const int hc = (warp - 2) >> 2;  // column half of this warp
     const int m = qd * 32 + lane;
     const int set = m >> 6, rr = m & 63;
+    const int ts = hc * 64 + rr;     // thread of the row set (0 .. 127)
     const RowSet* rs = set == 0 ? &ra : rb;
-    const int t128 = threadIdx.x - 64;
+    const int t256 = threadIdx.x - 64;
     // the tile's 128 query rows into the swizzled Q tile (16-byte copies, zero rows as padding)
-    for (int i = t128; i < 128 * 16; i += 128) {
+    for (int i = t256; i < 128 * 16; i += LQ_SOFTMAX) {
       const int r = i >> 4, c = i & 15;
       const RowSet* s_ = r < 64 ? &ra : rb;
       const int rl = r & 63;
@@ -266,68 +271,51 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
     const float sl2 = dp.scale * LOG2E;
     const bool k2d = tile.k_src == SRC_K2D;
     const int32_t* perm = k2d ? at<const int32_t>(dp, dp.lay.perm2d) : nullptr;
-    const uint32_t s_lane = tmem + ((uint32_t)(qd * 32) << 16);
+    const uint32_t s_lane = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(32 * hc);
 
-    // positions of the block's keys, warp-wide (modality-grouped keys: perm2d, else the row)
-    auto block_pos = [&](int64_t j0, int32_t& plo, int32_t& phi) -> int32_t {
-      if (!k2d) {
-        plo = (int32_t)(j0 + lane);
-        phi = plo + 32;
-        return (int32_t)(j0 + LQ_KB - 1);
-      }
-      plo = j0 + lane < dp.L ? __ldg(perm + j0 + lane) : 0x7fffffff;
-      phi = j0 + 32 + lane < dp.L ? __ldg(perm + j0 + 32 + lane) : 0x7fffffff;
-      int32_t mx = max(plo, phi);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-      return mx;
-    };
-    // the row's logits of block b in log2 units, -inf where the key is not causal
-    auto load_logits = [&](int b, float (&x)[64]) -> bool {
+    // the row's 32 logits of block b (this warp's column half) in log2 units, -inf where the key
+    // is not causal; key positions: modality-grouped keys through perm2d, else the row itself
+    auto load_logits = [&](int b, float (&x)[32]) -> bool {
       const int buf = b & 1;
-      const int64_t j0 = ck.c0 + (int64_t)b * LQ_KB;
-      int32_t plo, phi;
-      const int32_t bmax = block_pos(j0, plo, phi);
+      const int64_t j0 = ck.c0 + (int64_t)b * LQ_KB + 32 * hc;
+      int32_t pos, pmax;
+      if (!k2d) {
+        pos = (int32_t)(j0 + lane);
+        pmax = (int32_t)(j0 + 31);
+      } else {
+        pos = j0 + lane < dp.L ? __ldg(perm + j0 + lane) : 0x7fffffff;
+        pmax = pos;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pmax = max(pmax, __shfl_xor_sync(0xFFFFFFFFu, pmax, o));
+      }
       // the warp decides together (the loads below are warp-collective)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[buf], (b >> 1) & 1, abort))) return false;
       tc_fence_after();
-      // the row in two 32-column loads: the first half is scaled while the second is in flight
-      uint32_t sa[32], sb[32];
+      uint32_t sa[32];
       tmem_ld32(s_lane + (uint32_t)(buf * LQ_KB), sa);
       tmem_wait_ld_regs(sa);
-      tmem_ld32(s_lane + (uint32_t)(buf * LQ_KB + 32), sb);
-#pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sa[c]) * sl2;
-      tmem_wait_ld_regs(sb);
       tc_fence_before();
       mbar_arrive(&sm.s_free[buf]);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) x[32 + c] = __uint_as_float(sb[c]) * sl2;
-      if (__any_sync(0xFFFFFFFFu, bmax > pr)) {  // some key of the block is after some row of the warp
+      for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sa[c]) * sl2;
+      if (__any_sync(0xFFFFFFFFu, pmax > pr)) {  // some key of the half is after some row of the warp
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int32_t pos = __shfl_sync(0xFFFFFFFFu, c < 32 ? plo : phi, c & 31);
-          if (pos > pr) x[c] = -INFINITY;
-        }
+        for (int c = 0; c < 32; ++c)
+          if (__shfl_sync(0xFFFFFFFFu, pos, c) > pr) x[c] = -INFINITY;
       }
       return true;
     };
 
     if constexpr (PASS == 1) {
-      float mrun = -INFINITY, z = 0.f;
+      float mrun = -INFINITY, z = 0.f;  // over this thread's 32 columns of each block
       for (int b = 0; b < nblk; ++b) {
-        float x[64];
+        float x[32];
         if (!load_logits(b, x)) break;
-        // block max in eight independent chains of three-input maxima, then the sum of the
-        // exponentials in four chains (short dependency chains: the loop is latency-bound)
+        // the half-block max in eight independent chains, then the sum of the exponentials in
+        // four chains (short dependency chains: the loop is latency-bound)
         float m8[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) m8[q] = x[q];
-#pragma unroll
-        for (int c = 8; c < 64; c += 16) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) m8[q] = lq_fmax3(m8[q], x[c + q], x[c + 8 + q]);
-        }
+        for (int q = 0; q < 8; ++q) m8[q] = lq_fmax3(x[q], x[8 + q], fmaxf(x[16 + q], x[24 + q]));
         const float bm = fmaxf(lq_fmax3(m8[0], m8[1], m8[2]), lq_fmax3(m8[3], lq_fmax3(m8[4], m8[5], m8[6]), m8[7]));
         const float nm = fmaxf(mrun, bm);
         if (nm == -INFINITY) continue;
@@ -335,13 +323,27 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
         mrun = nm;
         float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) a[c & 3] += ex2(x[c] - mrun);
+        for (int c = 0; c < 32; ++c) a[c & 3] += ex2(x[c] - mrun);
         z += (a[0] + a[1]) + (a[2] + a[3]);
       }
-      if (rs != nullptr && chunk < rs->n_chunks) {
-        float* mz = at<float>(dp, rs->mz_off) + (int64_t)chunk * LASTQ * 2;
-        mz[2 * rr] = mrun;
-        mz[2 * rr + 1] = z;
+      // the two halves of each row: the second half's (max, sum) through shared memory, combined
+      // by the first half's thread (columns 0-31 first, then 32-63)
+      float* xch = reinterpret_cast<float*>(lq_smem + sizeof(Smem));
+      if (hc == 1) {
+        xch[2 * m] = mrun;
+        xch[2 * m + 1] = z;
+      }
+      asm volatile("bar.sync 3, %0;" ::"n"(LQ_SOFTMAX) : "memory");
+      if (hc == 0) {
+        const float m1 = xch[2 * m], z1 = xch[2 * m + 1];
+        const float M = fmaxf(mrun, m1);
+        float Z = 0.f;
+        if (M > -INFINITY) Z = (mrun > -INFINITY ? z * ex2(mrun - M) : 0.f) + (m1 > -INFINITY ? z1 * ex2(m1 - M) : 0.f);
+        if (rs != nullptr && chunk < rs->n_chunks) {
+          float* mz = at<float>(dp, rs->mz_off) + (int64_t)chunk * LASTQ * 2;
+          mz[2 * rr] = M;
+          mz[2 * rr + 1] = Z;
+        }
       }
     } else {
       LqtSmem2& s2 = *reinterpret_cast<LqtSmem2*>(lq_smem + sizeof(Smem));
@@ -359,9 +361,9 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
           max_rc = max(max_rc, c);
           contig = contig && c == rs->rcs[0] + r;
         }
-        s2.rcs[set][rr] = rr < rs->n_rows ? rs->rcs[rr] : 0;
+        if (hc == 0) s2.rcs[set][rr] = rr < rs->n_rows ? rs->rcs[rr] : 0;
       }
-      for (int i = rr; i < R; i += 64) ring[i] = 0.f;
+      for (int i = ts; i < R; i += 128) ring[i] = 0.f;
       const float* st = have ? at<const float>(dp, rs->stat_off) : nullptr;
       const float Mr = have ? st[2 * rr] : -INFINITY, Ir = have ? st[2 * rr + 1] : 0.f;
       const bool live = have && Mr > -INFINITY;
@@ -376,16 +378,16 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
 
       for (int b = 0; b < nblk; ++b) {
         const int64_t j0 = ck.c0 + (int64_t)b * LQ_KB;
-        float x[64];
+        float x[32];
         const bool got = load_logits(b, x);
         if (got) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) P[rr * P_PITCH + c] = live ? ex2(x[c] - Mr) * Ir : 0.f;
+          for (int c = 0; c < 32; ++c) P[rr * P_PITCH + 32 * hc + c] = live ? ex2(x[c] - Mr) * Ir : 0.f;
         }
         if (set_any(set, !got)) break;  // every thread of the set leaves together
-        // vertical sums of the keys the chunk owns: column rr, rows in a fixed order (four
-        // interleaved partial sums, so that the loads overlap)
-        {
+        if (hc == 0) {
+          // vertical sums of the keys the chunk owns: column rr, rows in a fixed order (four
+          // interleaved partial sums, so that the loads overlap)
           const int64_t j = j0 + rr;
           if (vout != nullptr && j >= own0 && j < own1) {
             float a[4] = {0.f, 0.f, 0.f, 0.f};
@@ -393,8 +395,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
             for (int r = 0; r < 64; ++r) a[r & 3] += P[r * P_PITCH + rr];
             vout[j] = (a[0] + a[1]) + (a[2] + a[3]);
           }
-        }
-        if (slash) {
+        } else if (slash) {
           const bool inside = j0 >= slo && j0 + LQ_KB <= shi;
           if (contig) {
             // consecutive row coordinates: offset rc0 - j0 + d collects diagonal d = r - c of the
@@ -431,7 +432,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
           }
         }
         set_sync(set);  // block's sums in the ring; P may be overwritten
-        if (slash) {
+        if (slash && hc == 0) {
           // offsets whose last-row key is j0 + rr are complete: written if the chunk owns them
           const int64_t o = (int64_t)max_rc - (j0 + rr);
           float& e = ring[o & (R - 1)];
@@ -504,7 +505,7 @@ bool lq_make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t heads, 
 
 // Shared memory the two passes launch with (pass 2 with `ring` slash-ring entries per row set).
 size_t lastq_smem_bytes(int pass, int ring) {
-  if (pass == 1) return sizeof(LqtSmem<1>);
+  if (pass == 1) return sizeof(LqtSmem<1>) + 2 * sizeof(float) * 128;  // + the row halves' exchange
   return sizeof(LqtSmem<2>) + sizeof(LqtSmem2) + 2 * sizeof(float) * (size_t)ring;
 }
 

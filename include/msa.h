@@ -323,7 +323,7 @@ msa_status msa_weight_share(const void* Q, const void* K, int64_t L, int32_t Hq,
  *    k_row_stride (elements, multiples of 8; pointers 16-byte aligned); softmax scale.
  *  - Outputs (device, caller-owned): v_out[k_v] vertical-line key positions and s_out[k_s]
  *    slash-line offsets, each ascending; counts_out[2] = number written to each.
- *  - Scratch: a fixed 1.1 MB array compiled into the library (every GPU that loads libmsa.so
+ *  - Scratch: a fixed 1.2 MB array compiled into the library (every GPU that loads libmsa.so
  *    holds it until the process exits); L must be a multiple of 64 and at most 65536, larger L
  *    returns MSA_ERR_UNSUPPORTED; k_v, k_s in [1, L].
  *  - The first call on a device looks up the array's device address (a runtime call, no
