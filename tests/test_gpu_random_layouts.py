@@ -4,7 +4,7 @@ at random.  Per layer: the device's index sets against the oracle's (near-tie ru
 and lse against the oracle's masked attention under the device's index sets, the device's count
 of allowed pairs against the oracle's masks (exact), and the index-based path bit-identical to
 the three-call path.  Every third layer runs with its keys cut into small chunks (the
-long-sequence path)."""
+long-sequence path); the Q-boundary heads of odd-numbered layers estimate per segment."""
 import numpy as np
 import pytest
 
@@ -42,7 +42,10 @@ def random_problem(seed: int) -> Problem:
         if k == "ashape":
             heads.append(Head(k, sink=int(rng.integers(0, 129)), local=int(rng.integers(1, 513))))
         elif k in ("vslash", "qbound", "bound2d"):
-            heads.append(Head(k, k_v=int(rng.integers(1, L // 4 + 1)), k_s=int(rng.integers(1, L // 2 + 1))))
+            # Q-boundary heads of odd-numbered layers estimate per segment (no extra draw, so the
+            # layers' other choices stay as they were)
+            heads.append(Head(k, k_v=int(rng.integers(1, L // 4 + 1)), k_s=int(rng.integers(1, L // 2 + 1)),
+                              per_segment=(k == "qbound" and seed % 2 == 1)))
         elif k == "block":
             if rng.random() < 0.5:
                 heads.append(Head(k, topk_blocks=int(rng.integers(1, 7))))
