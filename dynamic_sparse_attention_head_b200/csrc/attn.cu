@@ -774,12 +774,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       ItemInfo it;
       UnitInfo un;
       // units that skip their work touch no accumulator slot: counted finished at once
-      if (!load_unit(p, e, it, un) ||
-          (un.total > 0 && it.ntiles == 0) ||  // no keys of this item in this chunk
-          (un.total == 0 && un.chunk != 0)) {  // an item without tiles is written once
-        if (t == 0) band_unit_done(p, un);
-        continue;
-      }
+      if (!load_unit(p, e, it, un)) { if (t == 0) band_unit_done(p, un); continue; }
+      if (un.total > 0 && it.ntiles == 0) { if (t == 0) band_unit_done(p, un); continue; }  // no keys in this chunk
+      if (un.total == 0 && un.chunk != 0) { if (t == 0) band_unit_done(p, un); continue; }  // written once
       const ClassStatic& cs = class_of(p, it.cls);
       const int r = it.row0 + t;
       RowCtx& rc = sm.rctx[threadIdx.x - 128];
