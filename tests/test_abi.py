@@ -186,3 +186,24 @@ def _plan_with_cfg(p, cfg):
     h = ctypes.c_void_p()
     msa._check("msa_plan_create", msa._lib.msa_plan_create(ctypes.byref(pc), ctypes.byref(h)))
     msa._lib.msa_plan_destroy(h)
+
+
+def test_weight_share_argument_checks_come_before_any_device_access():
+    """msa_weight_share validates its arguments on the host (placeholder addresses, never
+    dereferenced) and returns at once for an empty sample."""
+    import ctypes
+    import dynamic_sparse_attention_head_b200 as msa
+    from dynamic_sparse_attention_head_b200 import Strides, _lib
+    s = Strides(q_head=131072 * 128, q_row=128, k_head=131072 * 128, k_row=128)
+    fake = 1 << 20  # 16-byte aligned, never touched
+    call = lambda Q=fake, K=fake, L=4096, Hq=4, Hkv=2, strides=ctypes.byref(s), scale=0.088, n=1, recall=0.95: \
+        _lib.msa_weight_share(Q, K, L, Hq, Hkv, strides, scale, fake, fake, n, recall, fake, None)  # noqa: E731
+    assert call(Q=None) == 1
+    assert call(recall=0.0) == 1 and call(recall=1.5) == 1
+    assert call(scale=0.0) == 1
+    assert call(n=-1) == 1
+    assert call(Hq=3) == 2  # Hq not a multiple of Hkv
+    assert call(Q=fake + 8) == 3  # misaligned
+    bad = Strides(q_head=131072 * 128, q_row=100, k_head=131072 * 128, k_row=128)
+    assert call(strides=ctypes.byref(bad)) == 3
+    assert call(n=0) == 0  # nothing to do: no launch
