@@ -312,9 +312,8 @@ msa_status msa_weight_share(const void* Q, const void* K, int64_t L, int32_t Hq,
 /* ---- allocation-free variant ----
  *
  * Vertical-slash index estimation of ONE query head (the vertical and slash lines of its last
- * 64 queries, by the rules msa_estimate applies to a vertical-slash head; its sums may be
- * rounded in another order, so at near-ties its lines may differ from msa_estimate's within
- * the tolerance both keep against an exact computation) for callers
+ * 64 queries, with the kernels, tile and key chunking msa_estimate uses for a one-head
+ * vertical-slash plan, so the lines are the same) for callers
  * that cannot allocate device memory or provide a workspace: code running inside another
  * framework's memory manager, or serving loops where cudaMalloc and its implicit device
  * synchronisation are not allowed.  This call has no counterpart in the method's description;

@@ -1,10 +1,10 @@
 """The allocation-free vertical-slash estimation (msa_vslash_estimate_static) serves callers
 that cannot allocate device memory or hand over a workspace (code running inside another
 framework's memory manager, serving loops where cudaMalloc and its device synchronisation are
-not allowed).  Its index sets must match the oracle's and the regular entry point's (msa_estimate
-on a one-head vertical-slash plan) under the near-tie rule, call after call: its scratch is one
-static array that every call reuses.  Collected last so a failure here comes after every other
-test has run."""
+not allowed).  Its index sets must match the oracle's under the near-tie rule and equal those of
+the regular entry point (msa_estimate on a one-head vertical-slash plan: the same kernels and key
+chunking), call after call: its scratch is one static array that every call reuses.  Collected
+last so a failure here comes after every other test has run."""
 import numpy as np
 import pytest
 
@@ -56,8 +56,8 @@ def test_static_scratch_matches_regular_entry_point_twice(L, k_v, k_s, seed):
         assert np.all(np.diff(V) > 0) and np.all(np.diff(S) > 0)
         near_tie_ok(V, orc["V"], orc["v"], what="vertical vs oracle")
         near_tie_ok(S, orc["S"], orc["s"], what="slash vs oracle")
-        near_tie_ok(V, ref["V"], orc["v"], what="vertical vs msa_estimate")
-        near_tie_ok(S, ref["S"], orc["s"], what="slash vs msa_estimate")
+        # the same sweep (one-head tile, same key chunks) as msa_estimate: the same lines
+        assert V.tolist() == ref["V"].tolist() and S.tolist() == ref["S"].tolist()
         if first is None:
             first = (V.tolist(), S.tolist())
         else:  # deterministic: the second call gives what the first gave
