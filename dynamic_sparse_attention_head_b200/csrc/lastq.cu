@@ -132,9 +132,50 @@ namespace {
 // row set's block, its rows' slash coordinates, and its slash ring (ring entries per set at
 // launch).
 struct LqtSmem2 {
-  float p[2][64 * P_PITCH];
+  float p[2][64 * P_PITCH];   // probabilities of row sets with non-consecutive coordinates
   int32_t rcs[2][64];
+  float vst[2][2][2][64];     // [block parity][set][row half][column]: column sums of a half
+  float dst[2][2][4][64];     // [block parity][set][quarter][diagonal + 32]: diagonal sums
 };
+
+// Butterfly reduce-scatter over the 32 lanes of a warp: lane l returns the sum over all lanes of
+// v[l], that is column l of the warp's 32 x 32 block (lane = row) summed over its rows, in a
+// fixed order.  Each step keeps the half of the columns named by one lane bit and adds the
+// partner lane's copy of it.
+__device__ __forceinline__ float warp_column_sums(const float (&v)[32], int lane) {
+  constexpr unsigned F = 0xFFFFFFFFu;
+  float a[16], b[8], c[4], d[2];
+  const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4, u2 = lane & 2, u1 = lane & 1;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a[i] = (u16 ? v[i + 16] : v[i]) + __shfl_xor_sync(F, u16 ? v[i] : v[i + 16], 16);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b[i] = (u8 ? a[i + 8] : a[i]) + __shfl_xor_sync(F, u8 ? a[i] : a[i + 8], 8);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = (u4 ? b[i + 4] : b[i]) + __shfl_xor_sync(F, u4 ? b[i] : b[i + 4], 4);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) d[i] = (u2 ? c[i + 2] : c[i]) + __shfl_xor_sync(F, u2 ? c[i] : c[i + 2], 2);
+  return (u1 ? d[1] : d[0]) + __shfl_xor_sync(F, u1 ? d[0] : d[1], 1);
+}
+
+// Diagonal sums of the warp's 32 x 32 block (lane = row r, register c = column): lane l returns
+// the sum along r - c = l in `hi` and along r - c = l - 32 in `lo` (empty for lane 0).  Step c
+// reads column c of row (l + c) mod 32, so every lane collects its diagonals in registers.
+__device__ __forceinline__ void warp_diagonal_sums(const float (&v)[32], int lane, float& hi, float& lo) {
+  float h0 = 0.f, h1 = 0.f, l0 = 0.f, l1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const float x = __shfl_sync(0xFFFFFFFFu, v[c], (lane + c) & 31);
+    if (lane + c < 32) {
+      if (c & 1) h1 += x;
+      else h0 += x;
+    } else {
+      if (c & 1) l1 += x;
+      else l0 += x;
+    }
+  }
+  hi = h0 + h1;
+  lo = l0 + l1;
+}
 
 // bar.red.or over the 128 threads of one row set: true if any of them passes true.
 template <int ID>
@@ -376,68 +417,85 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
       const int64_t own_end = ck.own0 + ra.chunk;  // offsets owned: last-row key in [own0, own_end)
       set_sync(set);  // ring and row coordinates in place
 
+      const int rh = rr >> 5;      // row half of the set held by this warp
+      const int w4 = rh * 2 + hc;  // the warp's quarter (row half, column half) of the set's block
+
       for (int b = 0; b < nblk; ++b) {
         const int64_t j0 = ck.c0 + (int64_t)b * LQ_KB;
-        float x[32];
-        const bool got = load_logits(b, x);
+        const int sb = b & 1;  // staging parity: a block's staging is rewritten two blocks later,
+                               // after every thread of the set has passed the barrier between
+        float p[32];
+        const bool got = load_logits(b, p);
         if (got) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) P[rr * P_PITCH + 32 * hc + c] = live ? ex2(x[c] - Mr) * Ir : 0.f;
+          for (int c = 0; c < 32; ++c) p[c] = live ? ex2(p[c] - Mr) * Ir : 0.f;
+          // vertical: column 32 hc + lane of the block summed over the warp's 32 rows
+          s2.vst[sb][set][rh][32 * hc + lane] = warp_column_sums(p, lane);
+          if (slash) {
+            if (!(j0 >= slo && j0 + LQ_KB <= shi)) {  // keys outside the slash range count zero
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const int64_t j = j0 + 32 * hc + c;
+                if (j < slo || j >= shi) p[c] = 0.f;
+              }
+            }
+            if (contig) {
+              float hi, lo;
+              warp_diagonal_sums(p, lane, hi, lo);
+              s2.dst[sb][set][w4][lane + 32] = hi;
+              s2.dst[sb][set][w4][lane] = lo;
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) P[rr * P_PITCH + 32 * hc + c] = p[c];
+            }
+          }
         }
         if (set_any(set, !got)) break;  // every thread of the set leaves together
-        if (hc == 0) {
-          // vertical sums of the keys the chunk owns: column rr, rows in a fixed order (four
-          // interleaved partial sums, so that the loads overlap)
-          const int64_t j = j0 + rr;
-          if (vout != nullptr && j >= own0 && j < own1) {
-            float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 16
-            for (int r = 0; r < 64; ++r) a[r & 3] += P[r * P_PITCH + rr];
-            vout[j] = (a[0] + a[1]) + (a[2] + a[3]);
+        // the set's 128 threads combine the four quarters in a fixed order
+        if (ts < 64) {
+          const int64_t j = j0 + ts;
+          if (vout != nullptr && j >= own0 && j < own1) vout[j] = s2.vst[sb][set][0][ts] + s2.vst[sb][set][1][ts];
+        }
+        if (slash && contig) {
+          // consecutive row coordinates: offset rc0 - j0 + d collects the block's diagonal
+          // d = r - c (-63 .. 63), held by quarter (h, c') at d - 32 (h - c'); thread ts takes
+          // d = ts - 64, adds it to the ring and writes the offset out once its last-row key is
+          // in this block
+          const int d = ts - 64;
+          float a = 0.f;
+          if (d >= -32 && d < 32) a += s2.dst[sb][set][0][d + 32];
+          if (d < 0) a += s2.dst[sb][set][1][d + 64];
+          if (d >= 0) a += s2.dst[sb][set][2][d];
+          if (d >= -32 && d < 32) a += s2.dst[sb][set][3][d + 32];
+          const int64_t o = rc0 - j0 + d;
+          float& e = ring[o & (R - 1)];
+          const float tot = e + a;
+          const int64_t kk = (int64_t)max_rc - o - j0;  // the offset's last-row key, from j0
+          if (kk >= 0 && kk < LQ_KB) {
+            if (j0 + kk >= own0 && j0 + kk < own_end && o >= 0 && o < dp.L) sout[o] = tot;
+            e = 0.f;
+          } else {
+            e = tot;
           }
         } else if (slash) {
-          const bool inside = j0 >= slo && j0 + LQ_KB <= shi;
-          if (contig) {
-            // consecutive row coordinates: offset rc0 - j0 + d collects diagonal d = r - c of the
-            // block; this thread sums diagonals rr - 63 (rows 0..rr) and rr + 1 (rows rr+1..63):
-            // row i contributes column (i + 63 - rr) mod 64 to one of the two (four interleaved
-            // partial sums each, combined in a fixed order)
-            float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 16
-            for (int i = 0; i < 64; ++i) {
-              const int c = (i + 63 - rr) & 63;
-              float v = P[i * P_PITCH + c];
-              if (!inside && (j0 + c < slo || j0 + c >= shi)) v = 0.f;
-              const bool lo = i <= rr;
-              a1[i & 3] += lo ? v : 0.f;
-              a2[i & 3] += lo ? 0.f : v;
+          // any row coordinates: one thread per offset touched by the block, rows in order
+          const int64_t olo = (int64_t)min_rc - (j0 + LQ_KB - 1), ohi = (int64_t)max_rc - j0;
+          for (int64_t o = olo + ts; o <= ohi; o += 128) {
+            float a = 0.f;
+            for (int r = 0; r < n_rows; ++r) {
+              const int64_t c = (int64_t)s2.rcs[set][r] - o - j0;
+              if (c >= 0 && c < LQ_KB) a += P[r * P_PITCH + (int)c];
             }
-            const float d1 = (a1[0] + a1[1]) + (a1[2] + a1[3]), d2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
-            const int64_t base = rc0 - j0;
-            ring[(base + rr - 63) & (R - 1)] += d1;
-            if (rr < 63) ring[(base + rr + 1) & (R - 1)] += d2;
-          } else {
-            // any row coordinates: one thread per offset touched by the block, rows in order
-            const int64_t olo = (int64_t)min_rc - (j0 + LQ_KB - 1), ohi = (int64_t)max_rc - j0;
-            for (int64_t o = olo + rr; o <= ohi; o += 64) {
-              float a = 0.f;
-              for (int r = 0; r < n_rows; ++r) {
-                const int64_t c = (int64_t)s2.rcs[set][r] - o - j0;
-                if (c < 0 || c >= LQ_KB) continue;
-                if (!inside && (j0 + c < slo || j0 + c >= shi)) continue;
-                a += P[r * P_PITCH + (int)c];
-              }
-              ring[o & (R - 1)] += a;
-            }
+            ring[o & (R - 1)] += a;
           }
-        }
-        set_sync(set);  // block's sums in the ring; P may be overwritten
-        if (slash && hc == 0) {
-          // offsets whose last-row key is j0 + rr are complete: written if the chunk owns them
-          const int64_t o = (int64_t)max_rc - (j0 + rr);
-          float& e = ring[o & (R - 1)];
-          if (j0 + rr >= own0 && j0 + rr < own_end && o >= 0 && o < dp.L) sout[o] = e;
-          e = 0.f;
+          set_sync(set);  // block's sums in the ring; P may be overwritten
+          if (ts < 64) {
+            // offsets whose last-row key is j0 + ts are complete: written if the chunk owns them
+            const int64_t o = (int64_t)max_rc - (j0 + ts);
+            float& e = ring[o & (R - 1)];
+            if (j0 + ts >= own0 && j0 + ts < own_end && o >= 0 && o < dp.L) sout[o] = e;
+            e = 0.f;
+          }
         }
       }
     }
