@@ -90,7 +90,7 @@ struct __align__(1024) Lq2Smem {
   uint64_t s_full[2], s_free[2], q_ready, drain;
   uint32_t tmem_base;
   int abort;
-  float m2[128];                    // per tile row: max + log2(normaliser), +inf: no probability
+  float nm2[128];                   // per tile row: -(max + log2(normaliser)), -inf: no probability
   int32_t pos[128];                 // per tile row: position (causal bound of its keys)
   int32_t rcs[128];                 // per tile row: slash coordinate
   float stg[2][2][4][P2_DIAG];      // [block parity][set][key quarter][entry]: diagonal sums
@@ -342,10 +342,13 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
     const int32_t* perm = k2d ? at<const int32_t>(dp, dp.lay.perm2d) : nullptr;
     const uint32_t s_lane = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(32 * hc);
 
-    float mrun = -INFINITY, z = 0.f;  // over this thread's 32 columns of each block
+    // over this thread's 32 columns of each block: running max of the raw logits, the same max
+    // in log2 units (mrun * sl2, the value every exponent is taken against) and the sum
+    float mrun = -INFINITY, ml2 = -INFINITY, z = 0.f;
+    const float2 sl2v = make_float2(sl2, sl2);
     for (int b = 0; b < nblk; ++b) {
-      // the row's 32 logits of block b (this warp's column half) in log2 units, -inf where the
-      // key is not causal; key positions: modality-grouped keys through perm2d, else the row
+      // the row's 32 raw logits of block b (this warp's column half), -inf where the key is not
+      // causal; key positions: modality-grouped keys through perm2d, else the row itself
       const int buf = b & 1;
       const int64_t j0 = ck.c0 + (int64_t)b * P1_KB + 32 * hc;
       int32_t pos, pmax;
@@ -368,27 +371,39 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
       mbar_arrive(&sm.s_free[buf]);
       float x[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sa[c]) * sl2;
+      for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sa[c]);
       if (__any_sync(0xFFFFFFFFu, pmax > pr)) {  // some key of the half is after some row of the warp
 #pragma unroll
         for (int c = 0; c < 32; ++c)
           if (__shfl_sync(0xFFFFFFFFu, pos, c) > pr) x[c] = -INFINITY;
       }
       // the half-block max in eight independent chains, then the sum of the exponentials in
-      // four chains (short dependency chains: the loop is latency-bound)
+      // pairs (short dependency chains: the loop is latency-bound)
       float m8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) m8[q] = lq_fmax3(x[q], x[8 + q], fmaxf(x[16 + q], x[24 + q]));
       const float bm = fmaxf(lq_fmax3(m8[0], m8[1], m8[2]), lq_fmax3(m8[3], lq_fmax3(m8[4], m8[5], m8[6]), m8[7]));
-      const float nm = fmaxf(mrun, bm);
-      if (nm == -INFINITY) continue;
-      z = (mrun == -INFINITY) ? 0.f : z * ex2(mrun - nm);
-      mrun = nm;
-      float a[4] = {0.f, 0.f, 0.f, 0.f};
+      if (!(bm > mrun)) {
+        if (mrun == -INFINITY) continue;  // nothing causal yet
+      } else {
+        const float nl2 = bm * sl2;
+        z = (mrun == -INFINITY) ? 0.f : z * ex2(ml2 - nl2);
+        mrun = bm;
+        ml2 = nl2;
+      }
+      const float2 neg = make_float2(-ml2, -ml2);
+      float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) a[c & 3] += ex2(x[c] - mrun);
-      z += (a[0] + a[1]) + (a[2] + a[3]);
+      for (int c = 0; c < 32; c += 4) {
+        const float2 t0 = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2v, neg);
+        const float2 t1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), sl2v, neg);
+        a0 = __fadd2_rn(a0, make_float2(ex2(t0.x), ex2(t0.y)));
+        a1 = __fadd2_rn(a1, make_float2(ex2(t1.x), ex2(t1.y)));
+      }
+      const float2 a = __fadd2_rn(a0, a1);
+      z += a.x + a.y;
     }
+    mrun = ml2;  // the row's max in log2 units from here on
     // the two halves of each row: the second half's (max, sum) through shared memory, combined
     // by the first half's thread (columns 0-31 first, then 32-63)
     if (hc == 1) {
@@ -418,21 +433,27 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
   }
 }
 
-// One half (32 query rows) of a pass-2 thread's key: the probabilities p = exp2(s * sl2 - m2)
-// (m2 = max + log2 Z of the row), their sum into va, and, with DIAG, the diagonals into lo / hi
-// (see diag_step).  With MASK: rows the key is not causal for count zero (key position kp after
-// the row's position), and so do all slash contributions of a key outside the slash range (dz).
-// The probabilities (zero outside the slash range) are left in sv for the caller.
+// One half (32 query rows) of a pass-2 thread's key: the probabilities p = exp2(s * sl2 + nm2)
+// (nm2 = -(max + log2 Z) of the row), their sum into va, and, with DIAG, the diagonals into
+// lo / hi (see diag_step).  With MASK: rows the key is not causal for count zero (key position
+// kp after the row's position), and so do all slash contributions of a key outside the slash
+// range (dz).  The probabilities (zero outside the slash range) are left in sv for the caller.
 template <bool MASK, bool DIAG>
-__device__ __forceinline__ void lq2_half(uint32_t (&sv)[32], const float* m2, const int32_t* pos, float sl2,
-                                         int32_t kp, bool dz, float (&va)[4], float& lo, float& hi) {
+__device__ __forceinline__ void lq2_half(uint32_t (&sv)[32], const float* nm2, const int32_t* pos, float2 sl2v,
+                                         int32_t kp, bool dz, float2 (&va)[2], float& lo, float& hi) {
   float p[32];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    float x = ex2(fmaf(__uint_as_float(sv[c]), sl2, -m2[c]));
-    if (MASK) x = kp > pos[c] ? 0.f : x;
-    va[c & 3] += x;
-    p[c] = MASK ? (dz ? 0.f : x) : x;
+  for (int c = 0; c < 32; c += 2) {
+    const float2 t = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2v,
+                                make_float2(nm2[c], nm2[c + 1]));
+    float x0 = ex2(t.x), x1 = ex2(t.y);
+    if (MASK) {
+      x0 = kp > pos[c] ? 0.f : x0;
+      x1 = kp > pos[c + 1] ? 0.f : x1;
+    }
+    va[(c >> 1) & 1] = __fadd2_rn(va[(c >> 1) & 1], make_float2(x0, x1));
+    p[c] = MASK && dz ? 0.f : x0;
+    p[c + 1] = MASK && dz ? 0.f : x1;
   }
   if (DIAG) DiagUnroll<32>::run(p, lo, hi);
 #pragma unroll
@@ -484,16 +505,16 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
     load_q_tile(sm.q, ra, rb, Q, qh, qr, t256);
     mbar_arrive(&sm.q_ready);
     if (t256 < 128) {
-      // per tile row: max + log2 Z from the pass-1 statistics, position, slash coordinate
+      // per tile row: -(max + log2 Z) from the pass-1 statistics, position, slash coordinate
       const int r = t256 & 63;
       const RowSet* s_ = t256 < 64 ? &ra : rb;
       const bool have = s_ != nullptr && r < s_->n_rows;
-      float m2 = INFINITY;
+      float nm2 = -INFINITY;
       if (have) {
         const float* st = at<const float>(dp, s_->stat_off);
-        if (st[2 * r] > -INFINITY) m2 = st[2 * r] + st[2 * r + 1];
+        if (st[2 * r] > -INFINITY) nm2 = -(st[2 * r] + st[2 * r + 1]);
       }
-      sm.m2[t256] = m2;
+      sm.nm2[t256] = nm2;
       sm.pos[t256] = have ? s_->rows[r] : -1;
       sm.rcs[t256] = have ? s_->rcs[r] : 0;
     }
@@ -525,7 +546,8 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
     const bool k2d = tile.k_src == SRC_K2D;
     const int32_t* perm = k2d ? at<const int32_t>(dp, dp.lay.perm2d) : nullptr;
     const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(64 * set);
-    const float* m2s = sm.m2 + 64 * set;
+    const float* m2s = sm.nm2 + 64 * set;
+    const float2 sl2v = make_float2(sl2, sl2);
     const int32_t* poss = sm.pos + 64 * set;
     const int32_t* rcss = sm.rcs + 64 * set;
     asm volatile("bar.sync 3, %0;" ::"n"(LQ_SOFTMAX) : "memory");  // tables and rings in place
@@ -538,7 +560,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
                              // the set has passed the barrier between
       // the warp decides together (the loads below are warp-collective)
       const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[buf], (b >> 1) & 1, abort));
-      float va[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 va[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       float d0 = 0.f, d1 = 0.f, d2 = 0.f;  // diagonals -32 q4 - lane, + 32, + 64 of the block
       if (ok) tc_fence_after();
       if (rs == nullptr) {
@@ -568,19 +590,19 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
             if (live) {
               float& lo = h == 0 ? d0 : d1;
               float& hi = h == 0 ? d1 : d2;
-              if (masked) lq2_half<true, true>(sv, m2h, posh, sl2, kp, dzero, va, lo, hi);
-              else lq2_half<false, true>(sv, m2h, posh, sl2, kp, dzero, va, lo, hi);
+              if (masked) lq2_half<true, true>(sv, m2h, posh, sl2v, kp, dzero, va, lo, hi);
+              else lq2_half<false, true>(sv, m2h, posh, sl2v, kp, dzero, va, lo, hi);
             }
           } else if (!slash) {
             if (live) {
-              if (masked) lq2_half<true, false>(sv, m2h, posh, sl2, kp, dzero, va, d0, d0);
-              else lq2_half<false, false>(sv, m2h, posh, sl2, kp, dzero, va, d0, d0);
+              if (masked) lq2_half<true, false>(sv, m2h, posh, sl2v, kp, dzero, va, d0, d0);
+              else lq2_half<false, false>(sv, m2h, posh, sl2v, kp, dzero, va, d0, d0);
             }
           } else {
             // any row coordinates: the set's four warps add their keys' slash values to the ring
             // in turn (within a warp the 32 keys of one row reach 32 distinct offsets), rows in
             // order; every warp of the set takes part in the barriers
-            if (live) lq2_half<true, false>(sv, m2h, posh, sl2, kp, dzero, va, d0, d0);
+            if (live) lq2_half<true, false>(sv, m2h, posh, sl2v, kp, dzero, va, d0, d0);
 #pragma unroll 1
             for (int qq = 0; qq < 4; ++qq) {
               set_sync(set);
@@ -590,7 +612,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
             }
           }
         }
-        if (live && k >= own0 && k < own1) vout[k] = (va[0] + va[1]) + (va[2] + va[3]);
+        if (live && k >= own0 && k < own1) vout[k] = (va[0].x + va[0].y) + (va[1].x + va[1].y);
         if (live && slash && contig) {
           sm.stg[sb][set][q4][lane] = d2;
           sm.stg[sb][set][q4][32 + lane] = d1;
