@@ -346,6 +346,13 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
     // in log2 units (mrun * sl2, the value every exponent is taken against) and the sum
     float mrun = -INFINITY, ml2 = -INFINITY, z = 0.f;
     const float2 sl2v = make_float2(sl2, sl2);
+    // modality-grouped keys: this lane's key position in block b, through perm2d (loaded one
+    // block ahead, so that the load overlaps the work on the block before)
+    auto grouped_pos = [&](int b) -> int32_t {
+      const int64_t j = ck.c0 + (int64_t)b * P1_KB + 32 * hc + lane;
+      return j < dp.L ? __ldg(perm + j) : 0x7fffffff;
+    };
+    int32_t pos_next = k2d && nblk > 0 ? grouped_pos(0) : 0;
     for (int b = 0; b < nblk; ++b) {
       // the row's 32 raw logits of block b (this warp's column half), -inf where the key is not
       // causal; key positions: modality-grouped keys through perm2d, else the row itself
@@ -356,7 +363,8 @@ __global__ void __launch_bounds__(LQ_THREADS, 2)
         pos = (int32_t)(j0 + lane);
         pmax = (int32_t)(j0 + 31);
       } else {
-        pos = j0 + lane < dp.L ? __ldg(perm + j0 + lane) : 0x7fffffff;
+        pos = pos_next;
+        if (b + 1 < nblk) pos_next = grouped_pos(b + 1);
         pmax = pos;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) pmax = max(pmax, __shfl_xor_sync(0xFFFFFFFFu, pmax, o));
