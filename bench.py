@@ -187,8 +187,12 @@ def job_totals(elapsed_ms: float, flops: float, world: int, device=None):
 
 
 # ---------------------------------------------------------------------------------------
-def make_host_inputs(p, seed):
-    Q, K, V = workload.make_inputs(p, seed=seed)
+INPUTS_NOTE = ("rope: N(0,1) rows plus a shared seeded direction of norm 9.5, rotated by the rotary "
+               "position embedding (base 1e6) of their position")
+
+
+def make_host_inputs(p, seed, inputs="iid"):
+    Q, K, V = workload.make_inputs(p, seed=seed, inputs=inputs)
     return Q, K, V
 
 
@@ -254,7 +258,7 @@ def measure_layer(args, name, rank, world, local_rank, steps, warmup, with_e2e, 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     p = workloads()[name]()
-    Qh, Kh, Vh = make_host_inputs(p, seed=rank)
+    Qh, Kh, Vh = make_host_inputs(p, seed=rank, inputs=args.inputs)
 
     def dev_copy(x):
         return torch.from_numpy(x).view(torch.bfloat16).to(dev)
@@ -463,6 +467,7 @@ def measure_layer(args, name, rank, world, local_rank, steps, warmup, with_e2e, 
         "value": value, "ms_per_step": ms_step, "ms_per_layer": ms_step, "steps": steps, "warmup": warmup,
         "config": {"workload": name, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
                    "heads": kind_summary(p), "parallelism": f"independent layer per rank x{world}",
+                   **({"inputs": INPUTS_NOTE} if args.inputs == "rope" else {}),
                    "l2": "inputs larger than L2 (no flush)" if (Qh.nbytes > 126e6) else "inputs smaller than L2",
                    "seed": "rank", **({"estimate_every": args.estimate_every} if args.estimate_every > 1 else {}),
                    **({"path": "index-based (Q rows gathered in the attention kernel, O written at "
@@ -564,7 +569,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     p = workloads()[args.workload]()
-    Qh, Kh, Vh = make_host_inputs(p, seed=0)
+    Qh, Kh, Vh = make_host_inputs(p, seed=0, inputs=args.inputs)
     flops = None
     # executed block FLOPs of the sampled heads' oracle indices, counted by the tile builder
     # (untimed, only to express the oracle's time in the metric's unit)
@@ -590,7 +595,7 @@ def run_reference(args, rank, world):
                             "from the oracle's own index sets) / the oracle's extrapolated layer time, so "
                             "that the ratio of the two arms' values is the ratio of their layer times"),
             "config": {"workload": args.workload, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
-                       "heads": kind_summary(p)},
+                       "heads": kind_summary(p), **({"inputs": INPUTS_NOTE} if args.inputs == "rope" else {})},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
                              "extrapolated": True, "sampled_rows_per_head": rows,
                              "sample": (f"per step: oracle on one head of each kind, full index estimation + "
@@ -625,6 +630,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="qwen2-7b-video-128k", choices=sorted(workloads()))
+    ap.add_argument("--inputs", choices=("iid", "rope"), default="iid",
+                    help="rope: Q/K rows with a shared component under the rotary position embedding, so that "
+                         "attention depends on the query-key offset (the index sets then cluster)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true",

@@ -48,6 +48,9 @@ def _load():
         lib.wl_normals_f64.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int64]
         lib.wl_fill_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64,
                                      ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float]
+        lib.wl_fill_rope_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64,
+                                          ctypes.c_uint64, ctypes.c_float, ctypes.c_void_p, ctypes.c_float,
+                                          ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float]
         _lib = lib
     return _lib
 
@@ -124,31 +127,51 @@ def frame_stride_rows(p: Problem, stride: int, phase: int = 0) -> np.ndarray:
 Q_STREAM, K_STREAM, V_STREAM, U_STREAM = 1000, 2000, 3000, 7
 
 
-def unit_vector(seed: int, d: int = 128) -> np.ndarray:
+def unit_vector(seed: int, d: int = 128, stream: int = U_STREAM) -> np.ndarray:
     lib = _load()
     u = np.empty(d, np.float64)
-    lib.wl_normals_f64(u.ctypes.data, d, seed, U_STREAM, 0)
+    lib.wl_normals_f64(u.ctypes.data, d, seed, stream, 0)
     return (u / np.linalg.norm(u)).astype(np.float32)
 
 
-def _fill(rows: int, d: int, seed: int, stream: int, bias=None, bias_rows=None, scale=0.0) -> np.ndarray:
+def _fill(rows: int, d: int, seed: int, stream: int, bias=None, bias_rows=None, scale=0.0, rope=None) -> np.ndarray:
     lib = _load()
     out = np.empty((rows, d), np.uint16)
     bptr = bias.ctypes.data if bias is not None else None
     rptr = bias_rows.ctypes.data if bias_rows is not None else None
-    lib.wl_fill_bf16(out.ctypes.data, rows, d, seed, stream, bptr, rptr, scale)
+    if rope is None:
+        lib.wl_fill_bf16(out.ctypes.data, rows, d, seed, stream, bptr, rptr, scale)
+    else:
+        shared, shared_scale, base = rope
+        lib.wl_fill_rope_bf16(out.ctypes.data, rows, d, seed, stream, 1.0, shared.ctypes.data, shared_scale, base,
+                              bptr, rptr, scale)
     return out
 
 
-def make_inputs(p: Problem, seed: int = 0, bias: float = 2.0, plant_queries: bool = False):
+# Position structure of the rotary variant: every Q and K row carries ROPE_SHARED x w (w a seeded
+# unit vector) before the rotary embedding of its position (base ROPE_BASE, the value of the
+# Qwen2 family), so q_i . k_j gains ROPE_SHARED^2 x w^T R(j - i) w, largest at offset 0 and
+# falling with distance: about 8 logits at offset 0 at the 1/sqrt(128) scale, against N(0, 1)
+# noise logits.
+ROPE_SHARED = 9.5
+ROPE_BASE = 1.0e6
+
+
+def make_inputs(p: Problem, seed: int = 0, bias: float = 2.0, plant_queries: bool = False, inputs: str = "iid"):
     """Q [Hq,L,d], K/V [Hkv,L,d] as bf16 bit patterns (np.uint16), head-major.
 
     K rows at frame-stride positions get ``bias * u`` when p.frame_stride > 0.
     With plant_queries, the last 64 video queries get the same shift, so the
     planted phase-0 grid dominates the last-64-query estimate.
+    inputs="rope": Q and K rows also carry the shared component of ROPE_SHARED and are rotated
+    by the rotary embedding of their position (V is unchanged), so that attention depends on the
+    offset between query and key as in a rotary model.
     """
+    if inputs not in ("iid", "rope"):
+        raise ValueError(f"inputs must be 'iid' or 'rope', not {inputs!r}")
     d = p.d
     u = unit_vector(seed, d)
+    rope = (unit_vector(seed, d, U_STREAM + 1), ROPE_SHARED, ROPE_BASE) if inputs == "rope" else None
     krows = None
     if p.frame_stride and bias:
         krows = frame_stride_rows(p, p.frame_stride).astype(np.uint8)
@@ -161,9 +184,9 @@ def make_inputs(p: Problem, seed: int = 0, bias: float = 2.0, plant_queries: boo
     K = np.empty((p.Hkv, p.L, d), np.uint16)
     V = np.empty((p.Hkv, p.L, d), np.uint16)
     for h in range(p.Hq):
-        Q[h] = _fill(p.L, d, seed, Q_STREAM + h, u if qrows is not None else None, qrows, bias)
+        Q[h] = _fill(p.L, d, seed, Q_STREAM + h, u if qrows is not None else None, qrows, bias, rope)
     for h in range(p.Hkv):
-        K[h] = _fill(p.L, d, seed, K_STREAM + h, u if krows is not None else None, krows, bias)
+        K[h] = _fill(p.L, d, seed, K_STREAM + h, u if krows is not None else None, krows, bias, rope)
         V[h] = _fill(p.L, d, seed, V_STREAM + h, None, None, 0.0)
     return Q, K, V
 

@@ -70,3 +70,39 @@ void wl_fill_bf16(uint16_t* out, int64_t rows, int32_t d, uint64_t seed, uint64_
     }
   }
 }
+
+/*
+ * Position-structured variant: row r is (noise_scale * N(0,1) + shared_scale * shared[c]
+ * [+ bias_scale * bias[c] on flagged rows]) rotated by the rotary position embedding of
+ * position r (Su et al., "RoFormer", 2021, in the half-split layout): dimensions m and
+ * m + d/2 form a pair rotated by the angle r * base^(-2m/d).  Dot products of two such rows then
+ * depend on their positions only through the offset between them, as in the rotary models the
+ * benchmark layers stand for.  Angles and rotations in double precision, rounded to fp32, then
+ * to bf16 (round to nearest even).
+ */
+void wl_fill_rope_bf16(uint16_t* out, int64_t rows, int32_t d, uint64_t seed, uint64_t stream,
+                       float noise_scale, const float* shared, float shared_scale, double base,
+                       const float* bias, const uint8_t* bias_rows, float bias_scale) {
+  const int32_t half = d / 2;
+  double freq[256];
+  if (d > 512) return;
+  for (int32_t m = 0; m < half; ++m) freq[m] = pow(base, -2.0 * (double)m / (double)d);
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    int add = bias && bias_rows && bias_rows[r];
+    float v[512];
+    for (int32_t c = 0; c < d; ++c) {
+      float x = noise_scale * (float)normal_at(seed, stream, (uint64_t)(r * d + c));
+      if (shared) x = x + shared_scale * shared[c];
+      if (add) x = x + bias_scale * bias[c];
+      v[c] = x;
+    }
+    for (int32_t m = 0; m < half; ++m) {
+      const double ang = (double)r * freq[m];
+      const double cs = cos(ang), sn = sin(ang);
+      const double a = v[m], b = v[m + half];
+      out[r * d + m] = f32_to_bf16_rne((float)(a * cs - b * sn));
+      out[r * d + m + half] = f32_to_bf16_rne((float)(a * sn + b * cs));
+    }
+  }
+}
