@@ -187,7 +187,7 @@ def job_totals(elapsed_ms: float, flops: float, world: int, device=None):
 
 
 # ---------------------------------------------------------------------------------------
-INPUTS_NOTE = ("rope: N(0,1) rows plus a shared seeded direction of norm 9.5, rotated by the rotary "
+INPUTS_NOTE = ("rope: N(0,1) rows plus a shared seeded direction of norm 15, rotated by the rotary "
                "position embedding (base 1e6) of their position")
 
 

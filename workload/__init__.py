@@ -151,9 +151,11 @@ def _fill(rows: int, d: int, seed: int, stream: int, bias=None, bias_rows=None, 
 # Position structure of the rotary variant: every Q and K row carries ROPE_SHARED x w (w a seeded
 # unit vector) before the rotary embedding of its position (base ROPE_BASE, the value of the
 # Qwen2 family), so q_i . k_j gains ROPE_SHARED^2 x w^T R(j - i) w, largest at offset 0 and
-# falling with distance: about 8 logits at offset 0 at the 1/sqrt(128) scale, against N(0, 1)
-# noise logits.
-ROPE_SHARED = 9.5
+# falling with distance (mean logits at the 1/sqrt(128) scale: ~20 at offset 0, ~15 at 100, ~9 at
+# 1000, ~4 at 4000).  The scale is set so that at 128K tokens a query needs about 2 % of its keys'
+# weights for 95 % of its attention mass, near the share the MMInference summary page reports for
+# VLM heads (1.79 %).
+ROPE_SHARED = 15.0
 ROPE_BASE = 1.0e6
 
 
