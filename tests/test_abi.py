@@ -207,3 +207,25 @@ def test_weight_share_argument_checks_come_before_any_device_access():
     bad = Strides(q_head=131072 * 128, q_row=100, k_head=131072 * 128, k_row=128)
     assert call(strides=ctypes.byref(bad)) == 3
     assert call(n=0) == 0  # nothing to do: no launch
+
+
+def test_estimation_rows_spanning_more_than_4096_positions_are_refused():
+    """The last 64 text queries of 4-token text runs between 316-token video runs span 4803
+    positions, above the 4096 the sweep's slash ring supports: plan creation says so."""
+    import numpy as np
+
+    import dynamic_sparse_attention_head_b200 as msa
+    from workload import TEXT, VIDEO, Head, Problem
+    segs, t = [], 0
+    for _ in range(17):
+        segs += [(t, 4, TEXT), (t + 4, 316, VIDEO)]
+        t += 320
+    p = Problem(L=t, Hq=1, Hkv=1, segments=segs, heads=[Head("qbound", k_v=8, k_s=16)], name="too-wide")
+    rows = np.nonzero(p.modality() == TEXT)[0][-64:]
+    assert rows[-1] - rows[0] > 4096
+    with pytest.raises(msa.MsaError) as e:
+        msa.Plan(p)
+    assert e.value.code == 5  # MSA_ERR_UNSUPPORTED
+    # a vertical-slash head on the same layout estimates from the last 64 positions (consecutive)
+    q = Problem(L=t, Hq=1, Hkv=1, segments=segs, heads=[Head("vslash", k_v=8, k_s=16)], name="vslash-only")
+    msa.Plan(q)
