@@ -6,7 +6,9 @@ msa_estimate -> msa_permute -> msa_sparse_prefill -> msa_unpermute.
 
 metric: sparse-prefill attention ms/layer + effective TFLOP/s (executed 128x128 block FLOPs,
 4 * 128^3 per tile) at 128K and 1M tokens.  `value` is effective TFLOP/s of the whole step,
-summed over ranks (each rank runs its own layer: weak scaling, no collective on the data path).
+summed over ranks (by default each rank runs its own layer: weak scaling; with --shard kv-heads
+the ranks split one layer by KV-head group: strong scaling; no collective on the data path in
+either).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 """
@@ -174,7 +176,7 @@ def cores():
 
 def job_totals(elapsed_ms: float, flops: float, world: int, device=None):
     """Max of the timed region over ranks and the sum of executed FLOPs over ranks (each rank
-    runs its own layer: weak scaling).  A collective only on these two scalars."""
+    runs its own layer or its own KV-head groups).  A collective only on these two scalars."""
     if world <= 1:
         return float(elapsed_ms), float(flops)
     import torch
@@ -258,7 +260,13 @@ def measure_layer(args, name, rank, world, local_rank, steps, warmup, with_e2e, 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     p = workloads()[name]()
-    Qh, Kh, Vh = make_host_inputs(p, seed=rank, inputs=args.inputs)
+    if args.shard == "kv-heads":
+        # one layer split by KV-head group: this rank's KV heads and their query heads, inputs
+        # drawn as those heads of the whole layer (one seed for all ranks)
+        p, qh, kvh = workload.shard_kv_heads(p, rank, world)
+        Qh, Kh, Vh = workload.make_inputs(p, seed=0, inputs=args.inputs, q_heads=qh, kv_heads=kvh)
+    else:
+        Qh, Kh, Vh = make_host_inputs(p, seed=rank, inputs=args.inputs)
 
     def dev_copy(x):
         return torch.from_numpy(x).view(torch.bfloat16).to(dev)
@@ -466,7 +474,10 @@ def measure_layer(args, name, rank, world, local_rank, steps, warmup, with_e2e, 
     return {
         "value": value, "ms_per_step": ms_step, "ms_per_layer": ms_step, "steps": steps, "warmup": warmup,
         "config": {"workload": name, "L": p.L, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d,
-                   "heads": kind_summary(p), "parallelism": f"independent layer per rank x{world}",
+                   "heads": kind_summary(p),
+                   "parallelism": (f"one layer split by KV-head group over {world} ranks ({p.Hkv} KV / {p.Hq} query "
+                                   f"heads per rank; per-head statistics on this line are rank 0's)"
+                                   if args.shard == "kv-heads" else f"independent layer per rank x{world}"),
                    **({"inputs": INPUTS_NOTE} if args.inputs == "rope" else {}),
                    "l2": "inputs larger than L2 (no flush)" if (Qh.nbytes > 126e6) else "inputs smaller than L2",
                    "seed": "rank", **({"estimate_every": args.estimate_every} if args.estimate_every > 1 else {}),
@@ -503,7 +514,8 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         line = {"metric": METRIC, "value": main.pop("value"), "unit": "TFLOP/s", "n_gpus": world,
                 "steps": main.pop("steps"), "warmup": main.pop("warmup"), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", **main}
+                "scaling": "strong" if args.shard == "kv-heads" else "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", **main}
         if second is not None:
             line["secondary"] = second
         print(json.dumps(line), flush=True)
@@ -633,6 +645,9 @@ def main():
     ap.add_argument("--inputs", choices=("iid", "rope"), default="iid",
                     help="rope: Q/K rows with a shared component under the rotary position embedding, so that "
                          "attention depends on the query-key offset (the index sets then cluster)")
+    ap.add_argument("--shard", choices=("layers", "kv-heads"), default="layers",
+                    help="layers: an independent layer per rank (weak scaling); kv-heads: one layer split by "
+                         "KV-head group over the ranks (strong scaling, no exchange)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true",

@@ -159,7 +159,8 @@ ROPE_SHARED = 15.0
 ROPE_BASE = 1.0e6
 
 
-def make_inputs(p: Problem, seed: int = 0, bias: float = 2.0, plant_queries: bool = False, inputs: str = "iid"):
+def make_inputs(p: Problem, seed: int = 0, bias: float = 2.0, plant_queries: bool = False, inputs: str = "iid",
+                q_heads: Optional[Sequence[int]] = None, kv_heads: Optional[Sequence[int]] = None):
     """Q [Hq,L,d], K/V [Hkv,L,d] as bf16 bit patterns (np.uint16), head-major.
 
     K rows at frame-stride positions get ``bias * u`` when p.frame_stride > 0.
@@ -168,6 +169,8 @@ def make_inputs(p: Problem, seed: int = 0, bias: float = 2.0, plant_queries: boo
     inputs="rope": Q and K rows also carry the shared component of ROPE_SHARED and are rotated
     by the rotary embedding of their position (V is unchanged), so that attention depends on the
     offset between query and key as in a rotary model.
+    q_heads / kv_heads: draw only these heads of a larger layer (their streams keep the layer's
+    head numbers, so a shard's inputs equal the same heads of the whole layer's).
     """
     if inputs not in ("iid", "rope"):
         raise ValueError(f"inputs must be 'iid' or 'rope', not {inputs!r}")
@@ -182,15 +185,33 @@ def make_inputs(p: Problem, seed: int = 0, bias: float = 2.0, plant_queries: boo
         vid = np.nonzero(p.modality() == VIDEO)[0]
         qrows = np.zeros(p.L, np.uint8)
         qrows[vid[-64:]] = 1
-    Q = np.empty((p.Hq, p.L, d), np.uint16)
-    K = np.empty((p.Hkv, p.L, d), np.uint16)
-    V = np.empty((p.Hkv, p.L, d), np.uint16)
-    for h in range(p.Hq):
-        Q[h] = _fill(p.L, d, seed, Q_STREAM + h, u if qrows is not None else None, qrows, bias, rope)
-    for h in range(p.Hkv):
-        K[h] = _fill(p.L, d, seed, K_STREAM + h, u if krows is not None else None, krows, bias, rope)
-        V[h] = _fill(p.L, d, seed, V_STREAM + h, None, None, 0.0)
+    qs = list(range(p.Hq)) if q_heads is None else list(q_heads)
+    ks = list(range(p.Hkv)) if kv_heads is None else list(kv_heads)
+    Q = np.empty((len(qs), p.L, d), np.uint16)
+    K = np.empty((len(ks), p.L, d), np.uint16)
+    V = np.empty((len(ks), p.L, d), np.uint16)
+    for i, h in enumerate(qs):
+        Q[i] = _fill(p.L, d, seed, Q_STREAM + h, u if qrows is not None else None, qrows, bias, rope)
+    for i, h in enumerate(ks):
+        K[i] = _fill(p.L, d, seed, K_STREAM + h, u if krows is not None else None, krows, bias, rope)
+        V[i] = _fill(p.L, d, seed, V_STREAM + h, None, None, 0.0)
     return Q, K, V
+
+
+def shard_kv_heads(p: Problem, rank: int, world: int) -> Tuple[Problem, range, range]:
+    """Rank `rank`'s share of one layer split by KV-head group over `world` GPUs: KV heads
+    [rank Hkv/world, (rank + 1) Hkv/world) and the query heads that read them (query head h reads
+    KV head h // (Hq / Hkv)).  Heads are independent in every step of the path, so the shards
+    need no exchange; returns (sub-problem, query heads, KV heads) in the full layer's numbering."""
+    if world < 1 or not 0 <= rank < world or p.Hkv % world:
+        raise ValueError(f"{p.Hkv} KV heads do not split over {world} ranks")
+    nkv = p.Hkv // world
+    nq = p.Hq // world
+    qh = range(rank * nq, (rank + 1) * nq)
+    kvh = range(rank * nkv, (rank + 1) * nkv)
+    sub = Problem(L=p.L, Hq=nq, Hkv=nkv, segments=list(p.segments), heads=[p.heads[h] for h in qh], d=p.d,
+                  name=f"{p.name}[kv {kvh.start}-{kvh.stop - 1}]", frame_stride=p.frame_stride, scale=p.scale)
+    return sub, qh, kvh
 
 
 def bf16_to_f32(x: np.ndarray) -> np.ndarray:
