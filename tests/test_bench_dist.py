@@ -40,6 +40,38 @@ def test_job_totals_two_gloo_ranks():
     assert res[0] == res[1] == (15.0, 3e12)
 
 
+def _shard_worker(rank, world, port, out):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch
+    import workload
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        p = workload.qwen2_7b_video_128k()
+        sub, qh, kvh = workload.shard_kv_heads(p, rank, world)
+        mine = torch.tensor(list(qh) + [-1] * (p.Hq - len(qh)), dtype=torch.int64)
+        parts = [torch.empty_like(mine) for _ in range(world)]
+        dist.all_gather(parts, mine)
+        out[rank] = sorted(int(h) for t in parts for h in t.tolist() if h >= 0), (sub.Hq, sub.Hkv)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_kv_head_shards_of_two_gloo_ranks_cover_the_layer():
+    """Each of two ranks takes its KV-head groups of the 128K layer (14 query / 2 KV heads); the
+    union over ranks is every query head exactly once."""
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        mp.start_processes(_shard_worker, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
+        res = dict(out)
+    assert res[0][0] == res[1][0] == list(range(28))
+    assert res[0][1] == res[1][1] == (14, 2)
+
+
 def test_job_totals_single_rank_is_identity():
     import sys
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
