@@ -454,6 +454,18 @@ __device__ __forceinline__ void mark_units(uint32_t* bm, int64_t a, int64_t b, i
   }
 }
 
+// Window starts of one bitmap word for the greedy cover (see tiles_kernel): the marked units at
+// an even distance from the start of their run; cin: the first unit is covered by the window
+// before the word.  Runs that start at even positions are found by adding their start bits (the
+// carry clears exactly the run).
+__device__ __forceinline__ uint32_t window_starts(uint32_t x, uint32_t cin) {
+  if (cin) x &= ~1u;
+  const uint32_t even = 0x55555555u;
+  const uint32_t rs = x & ~(x << 1);              // run starts
+  const uint32_t re = x & ~(x + (rs & even));     // units of runs that start at even positions
+  return (re & even) | (x & ~re & ~even);
+}
+
 __global__ void __launch_bounds__(TB_WARPS * 32) tiles_kernel(DevPlan dp, int bm_words) {
   extern __shared__ uint32_t tb_smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -567,33 +579,67 @@ __global__ void __launch_bounds__(TB_WARPS * 32) tiles_kernel(DevPlan dp, int bm
       }
     }
     __syncwarp();
-    // ---- greedy cover of the marked units by disjoint 2-unit windows (lane 0)
-    if (lane == 0) {
-      int carry = 0;
-      for (int w = 0; w < wmax; ++w) {
-        uint32_t x = bm[w];
-        if (carry) x &= ~1u;
-        carry = 0;
-        while (x) {
-          const int b = __ffs(x) - 1;
-          const int64_t u = ((int64_t)w << 5) + b;
-          if (nt < cs.tile_cap) out[nt] = ((uint32_t)cs.k_src << 28) | (uint32_t)(cs.krow_lo + u * UNIT);
-          ++nt;
-          if (b == 31) {
-            carry = 1;
-            x = 0;
-          } else {
-            x &= ~(3u << b);
-          }
+    // ---- greedy cover of the marked units by disjoint 2-unit windows, scanning units upwards: a
+    // window starts at every marked unit not covered by the window before it, which is every
+    // marked unit at an even distance from the start of its run of marked units.  Each lane
+    // takes a run of words; the one bit of state between words (the last window covers the next
+    // word's first unit) goes across the lanes by a scan of the words' carry maps.
+    {
+      const int per = (wmax + 31) >> 5;
+      const int w0 = min(lane * per, wmax), w1 = min(w0 + per, wmax);
+      uint32_t f0 = 0u, f1 = 1u;  // carry out of this lane's words for carry in 0 / 1
+      for (int w = w0; w < w1; ++w) {
+        const uint32_t x = bm[w];
+        f0 = window_starts(x, f0) >> 31;
+        f1 = window_starts(x, f1) >> 31;
+      }
+      // inclusive scan of the maps (composition: earlier lanes' map first)
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t g0 = __shfl_up_sync(0xFFFFFFFFu, f0, o), g1 = __shfl_up_sync(0xFFFFFFFFu, f1, o);
+        if (lane >= o) {
+          const uint32_t h0 = g0 ? f1 : f0, h1 = g1 ? f1 : f0;
+          f0 = h0;
+          f1 = h1;
         }
       }
-      if (nt > cs.tile_cap) {
-        flag_bounds(dp);
-        nt = cs.tile_cap;
+      uint32_t cin = __shfl_up_sync(0xFFFFFFFFu, f0, 1);  // the chain starts with carry 0
+      if (lane == 0) cin = 0u;
+      // windows of this lane's words, then their places in the list
+      int cnt = 0;
+      uint32_t c = cin;
+      for (int w = w0; w < w1; ++w) {
+        const uint32_t st = window_starts(bm[w], c);
+        c = st >> 31;
+        cnt += __popc(st);
       }
-      ntiles[item] = nt;
+      int base = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, base, o);
+        if (lane >= o) base += v;
+      }
+      const int total = __shfl_sync(0xFFFFFFFFu, base, 31);
+      base = nt + base - cnt;
+      c = cin;
+      for (int w = w0; w < w1; ++w) {
+        uint32_t st = window_starts(bm[w], c);
+        c = st >> 31;
+        while (st) {
+          const int b = __ffs(st) - 1;
+          st &= st - 1u;
+          const int64_t u = ((int64_t)w << 5) + b;
+          if (base < cs.tile_cap) out[base] = ((uint32_t)cs.k_src << 28) | (uint32_t)(cs.krow_lo + u * UNIT);
+          ++base;
+        }
+      }
+      nt += total;
+      if (lane == 0) {
+        if (nt > cs.tile_cap) flag_bounds(dp);
+        ntiles[item] = min(nt, cs.tile_cap);
+      }
+      nt = min(nt, cs.tile_cap);
     }
-    nt = __shfl_sync(0xFFFFFFFFu, min(nt, cs.tile_cap), 0);
     __syncwarp();
     // ---- tiles that every row of the item attends to in full (sufficient conditions only)
     const int32_t qpos_min = pos_of(row0);
