@@ -134,7 +134,7 @@ const char* msa_status_string(msa_status s) {
     case MSA_ERR_SHAPE: return "bad shape (d must be 128, L a multiple of 64, Hq a multiple of Hkv, segments tiling [0, L))";
     case MSA_ERR_ALIGN: return "misaligned pointer or stride (16-byte pointers, strides multiple of 8 elements, 256-byte workspace)";
     case MSA_ERR_WORKSPACE: return "workspace smaller than msa_workspace_bytes()";
-    case MSA_ERR_UNSUPPORTED: return "outside this build's limits (L < 2^27, grid stride <= 4096, estimation rows spanning <= 8192 positions)";
+    case MSA_ERR_UNSUPPORTED: return "outside this build's limits (L < 2^27, grid stride <= 4096, estimation rows spanning <= 4096 positions)";
     case MSA_ERR_CUDA: return "CUDA call failed";
     case MSA_ERR_TIMEOUT: return "device: a bounded wait expired";
     case MSA_ERR_DEVICE_BOUNDS: return "device: an index fell outside its buffer";
