@@ -366,9 +366,9 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
           if (s < C[c].n_items) P->items.push_back(WorkItem{c, s});
     }
     // ---- key chunks of the attention kernel: when one head's K and V (L x 512 B) no longer fit
-    // comfortably in L2, the keys are cut into 64K-key chunks (32 MB of K and V per head); the
+    // comfortably in L2, the keys are cut into 128K-key chunks (64 MB of K and V per head); the
     // environment variable MSA_ATTN_CHUNK_KEYS (a multiple of 128) overrides the chunk size.
-    int64_t ck = (int64_t)L * 512 > (96ll << 20) ? 65536 : 0;
+    int64_t ck = (int64_t)L * 512 > (96ll << 20) ? 131072 : 0;
     if (const char* env = std::getenv("MSA_ATTN_CHUNK_KEYS")) ck = std::max<int64_t>(0, std::atoll(env)) / TILE * TILE;
     P->n_kchunks = (ck > 0 && ck < L) ? (int32_t)((L + ck - 1) / ck) : 1;
     P->chunk_keys = P->n_kchunks > 1 ? (int32_t)ck : (int32_t)L;

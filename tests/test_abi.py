@@ -76,14 +76,14 @@ def test_indexed_workspace_drops_the_permuted_copies():
 
 
 def test_attention_units_chunking_rule(monkeypatch):
-    """Keys are chunked (65536 per chunk) only when one head's K and V exceed ~96 MB; the
+    """Keys are chunked (131072 per chunk) only when one head's K and V exceed ~96 MB; the
     environment override applies at plan creation."""
     import dynamic_sparse_attention_head_b200 as msa
     import workload
     monkeypatch.delenv("MSA_ATTN_CHUNK_KEYS", raising=False)
     assert msa.Plan(workload.qwen2_7b_video_128k()).attention_units()[1] == 1
     units, chunks = msa.Plan(workload.longvila_1m()).attention_units()
-    assert chunks == 16
+    assert chunks == 8
     monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", "256")
     p = workload.llama3_8b_text(L=2048)
     assert msa.Plan(p).attention_units()[1] == 8
