@@ -277,126 +277,177 @@ __global__ void grid_detect_kernel(DevPlan dp) {
 }
 
 // ---------------------------------------------------------------------------------------
-// grid classes: marks, row lists of both classes, gathered grid keys, exclusion bitmap.
-// One CTA (1024 threads) per grid head; each thread owns a contiguous run of positions
-// whose length is a multiple of 32 so bitmap words are written without atomics.
+// grid classes: row lists of both classes, gathered grid keys, exclusion bitmap.
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ int block_excl_scan(int x, int* sh, int* total) {
-  // 1024 threads; sh holds 32 ints
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int v = x;
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xFFFFFFFFu, v, o);
-    if (lane >= o) v += y;
-  }
-  if (lane == 31) sh[w] = v;
-  __syncthreads();
-  if (w == 0) {
-    int s = sh[lane];
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xFFFFFFFFu, s, o);
-      if (lane >= o) s += y;
-    }
-    sh[lane] = s;  // inclusive over warps
-  }
-  __syncthreads();
-  const int before_warp = w ? sh[w - 1] : 0;
-  *total = sh[31];
-  __syncthreads();
-  return before_warp + v - x;
-}
 
-__global__ void __launch_bounds__(1024) grid_mat_kernel(DevPlan dp) {
-  const int h = blockIdx.x;
-  const HeadStatic& hs = head(dp, h);
-  if (hs.kind != MSA_GRID) return;
-  __shared__ uint32_t pset[128];  // phase bitmap, strides <= 4096
-  __shared__ int scan_sh[32];
+// Grid heads, materialised in two launches over GM_BLOCKS blocks per head (each block a run of
+// whole 32-position words): positions whose in-segment offset mod the stride is one of the
+// selected phases (video only) are the gathered keys of the head's video class and excluded from
+// its identity tiles; query rows split into class 0 (text rows and those grid positions) and
+// class 1 (the other video rows), all lists in ascending position order.
+constexpr int GM_BLOCKS = 32;
+constexpr int GM_THREADS = 256;
+
+struct GridCtx {
+  int s, np;
+  int64_t b0, b1;  // this block's positions
+};
+
+// The block's positions and the phase bitmap of the head (shared memory); false: not a grid head.
+__device__ __forceinline__ bool grid_block(const DevPlan& dp, const HeadStatic& hs, uint32_t* pset, GridCtx& g) {
+  if (hs.kind != MSA_GRID) return false;
   const int32_t* counts = at<const int32_t>(dp, hs.counts_off);
-  const int s = counts[6], np = counts[7];
+  g.s = counts[6];
+  g.np = counts[7];
   const int32_t* phases = at<const int32_t>(dp, hs.phases_off);
   for (int i = threadIdx.x; i < 128; i += blockDim.x) pset[i] = 0u;
   __syncthreads();
-  if (threadIdx.x < np) {
-    const int ph = phases[threadIdx.x];
+  for (int i = threadIdx.x; i < g.np; i += blockDim.x) {
+    const int ph = phases[i];
     if (ph >= 0 && ph < 4096) atomicOr(&pset[ph >> 5], 1u << (ph & 31));
   }
   __syncthreads();
-  const ClassStatic& c0 = cls(dp, hs.class0);
-  const ClassStatic& c1 = cls(dp, hs.class0 + 1);
-  const int64_t L = dp.L;
-  const int64_t per = ((L + blockDim.x - 1) / blockDim.x + 31) / 32 * 32;
-  const int64_t t0 = min((int64_t)threadIdx.x * per, L), t1 = min(t0 + per, L);
-  const uint8_t* mod = at<const uint8_t>(dp, dp.lay.modality);
-  const int32_t* seg = at<const int32_t>(dp, dp.lay.segs);
-  uint8_t* gm = at<uint8_t>(dp, hs.gmark_off);
-  // pass 1: marks and counts
-  int g_cnt = 0, c0_cnt = 0, c1_cnt = 0;
-  {
-    int sidx = 0;
-    // first segment overlapping t0
-    int lo = 0, hi = dp.n_segs - 1;
-    while (lo < hi) {
-      int m = (lo + hi + 1) >> 1;
-      if (seg[3 * m] <= t0) lo = m;
-      else hi = m - 1;
-    }
-    sidx = lo;
-    for (int64_t t = t0; t < t1; ++t) {
-      while (sidx + 1 < dp.n_segs && seg[3 * (sidx + 1)] <= t) ++sidx;
-      uint8_t g = 0;
-      if (mod[t] == MSA_VIDEO) {
-        const int ph = (int)((t - seg[3 * sidx]) % s);
-        g = (pset[ph >> 5] >> (ph & 31)) & 1u;
+  const int64_t words = (dp.L + 31) >> 5;
+  const int64_t per = (words + GM_BLOCKS - 1) / GM_BLOCKS;
+  g.b0 = min((int64_t)blockIdx.x * per, words) << 5;
+  g.b1 = min(((int64_t)blockIdx.x + 1) * per, words) << 5;
+  return true;
+}
+
+// One 32-position word of a block (lane = position t = w0 + lane): the grid mark and the class.
+// Returns ballots: marks, class-0 rows, class-1 rows.
+__device__ __forceinline__ void grid_word(const DevPlan& dp, const uint32_t* pset, int s, int64_t w0, uint32_t& gb,
+                                          uint32_t& c0b, uint32_t& c1b) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = w0 + lane;
+  const bool valid = t < dp.L;
+  bool g = false, text = false;
+  if (valid) {
+    const uint8_t m = at<const uint8_t>(dp, dp.lay.modality)[t];
+    text = m == MSA_TEXT;
+    if (m == MSA_VIDEO) {
+      // segment of t: the last whose start is <= t
+      const int32_t* seg = at<const int32_t>(dp, dp.lay.segs);
+      int lo = 0, hi = dp.n_segs - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (seg[3 * mid] <= t) lo = mid;
+        else hi = mid - 1;
       }
-      gm[t] = g;
-      g_cnt += g;
-      if (g || mod[t] == MSA_TEXT) ++c0_cnt;
-      else ++c1_cnt;
+      const int ph = (int)((t - seg[3 * lo]) % s);
+      g = (pset[ph >> 5] >> (ph & 31)) & 1u;
     }
   }
+  gb = __ballot_sync(0xFFFFFFFFu, g);
+  c0b = __ballot_sync(0xFFFFFFFFu, valid && (g || text));
+  c1b = __ballot_sync(0xFFFFFFFFu, valid && !(g || text));
+}
+
+// Pass 1: per block, the number of grid marks, class-0 rows and class-1 rows.
+__global__ void __launch_bounds__(GM_THREADS) grid_count_kernel(DevPlan dp) {
+  const HeadStatic& hs = head(dp, blockIdx.y);
+  __shared__ uint32_t pset[128];  // phase bitmap, strides <= 4096
+  __shared__ int sums[GM_THREADS / 32][3];
+  GridCtx g;
+  if (!grid_block(dp, hs, pset, g)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  int n[3] = {0, 0, 0};
+  for (int64_t w0 = g.b0 + 32 * warp; w0 < g.b1; w0 += 32 * nw) {
+    uint32_t gb, c0b, c1b;
+    grid_word(dp, pset, g.s, w0, gb, c0b, c1b);
+    n[0] += __popc(gb);
+    n[1] += __popc(c0b);
+    n[2] += __popc(c1b);
+  }
+  if (lane == 0)
+    for (int i = 0; i < 3; ++i) sums[warp][i] = n[i];
   __syncthreads();
-  int g_tot, c0_tot, c1_tot;
-  const int g_off = block_excl_scan(g_cnt, scan_sh, &g_tot);
-  const int c0_off = block_excl_scan(c0_cnt, scan_sh, &c0_tot);
-  const int c1_off = block_excl_scan(c1_cnt, scan_sh, &c1_tot);
-  if (g_tot > c1.x_cap) {
+  if (threadIdx.x < 3) {
+    int v = 0;
+    for (int w = 0; w < nw; ++w) v += sums[w][threadIdx.x];
+    at<int32_t>(dp, hs.counts_off)[16 + 3 * blockIdx.x + threadIdx.x] = v;
+  }
+}
+
+// Pass 2: each block writes its marks, rows and exclusion words at the offsets of the blocks
+// before it; warps take consecutive runs of words, so every list stays in position order.
+__global__ void __launch_bounds__(GM_THREADS) grid_write_kernel(DevPlan dp) {
+  const int h = blockIdx.y;
+  const HeadStatic& hs = head(dp, h);
+  __shared__ uint32_t pset[128];
+  __shared__ int wsum[GM_THREADS / 32][3];
+  __shared__ int base[3], tot[3];
+  GridCtx g;
+  if (!grid_block(dp, hs, pset, g)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int32_t* bc = at<const int32_t>(dp, hs.counts_off) + 16;
+  if (threadIdx.x < 3) {
+    int before = 0, all = 0;
+    for (int b = 0; b < GM_BLOCKS; ++b) {
+      const int v = bc[3 * b + threadIdx.x];
+      if (b < (int)blockIdx.x) before += v;
+      all += v;
+    }
+    base[threadIdx.x] = before;
+    tot[threadIdx.x] = all;
+  }
+  // this warp's run of words
+  const int64_t nwords = (g.b1 - g.b0) >> 5;
+  const int64_t wper = (nwords + nw - 1) / nw;
+  const int64_t wa = g.b0 + 32 * min((int64_t)warp * wper, nwords), wb = g.b0 + 32 * min((int64_t)(warp + 1) * wper, nwords);
+  int n[3] = {0, 0, 0};
+  for (int64_t w0 = wa; w0 < wb; w0 += 32) {
+    uint32_t gb, c0b, c1b;
+    grid_word(dp, pset, g.s, w0, gb, c0b, c1b);
+    n[0] += __popc(gb);
+    n[1] += __popc(c0b);
+    n[2] += __popc(c1b);
+  }
+  if (lane == 0)
+    for (int i = 0; i < 3; ++i) wsum[warp][i] = n[i];
+  __syncthreads();
+  const ClassStatic& c0 = cls(dp, hs.class0);
+  const ClassStatic& c1 = cls(dp, hs.class0 + 1);
+  if (tot[0] > c1.x_cap) {
     if (threadIdx.x == 0) flag_bounds(dp);
     return;
+  }
+  int off[3];
+  for (int i = 0; i < 3; ++i) {
+    off[i] = base[i];
+    for (int w = 0; w < warp; ++w) off[i] += wsum[w][i];
   }
   int32_t* rows0 = at<int32_t>(dp, c0.rows_off);
   int32_t* rows1 = at<int32_t>(dp, c1.rows_off);
   int32_t* xg = at<int32_t>(dp, c1.x_pos_off);
   uint32_t* ex = at<uint32_t>(dp, c1.excl_bits_off);
-  {
-    int gi = g_off, i0 = c0_off, i1 = c1_off;
-    uint32_t word = 0u;
-    for (int64_t t = t0; t < t1; ++t) {
-      const uint8_t g = gm[t];
-      if (g) {
-        xg[gi++] = (int32_t)t;
-        word |= 1u << (t & 31);
-      }
-      if (g || mod[t] == MSA_TEXT) rows0[i0++] = (int32_t)t;
-      else rows1[i1++] = (int32_t)t;
-      if ((t & 31) == 31 || t == t1 - 1) {
-        ex[t >> 5] = word;
-        word = 0u;
-      }
-    }
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int64_t w0 = wa; w0 < wb; w0 += 32) {
+    uint32_t gb, c0b, c1b;
+    grid_word(dp, pset, g.s, w0, gb, c0b, c1b);
+    const int64_t t = w0 + lane;
+    if ((gb >> lane) & 1u) xg[off[0] + __popc(gb & lt)] = (int32_t)t;
+    if ((c0b >> lane) & 1u) rows0[off[1] + __popc(c0b & lt)] = (int32_t)t;
+    if ((c1b >> lane) & 1u) rows1[off[2] + __popc(c1b & lt)] = (int32_t)t;
+    if (lane == 0) ex[w0 >> 5] = gb;
+    off[0] += __popc(gb);
+    off[1] += __popc(c0b);
+    off[2] += __popc(c1b);
   }
-  for (int i = g_tot + threadIdx.x; i < c1.x_cap; i += blockDim.x) xg[i] = POS_PAD;
-  if (threadIdx.x == 0) {
-    ClassDyn& d0 = dyn(dp, c0.dyn);
-    d0.nrows = c0_tot;
-    d0.qrow0 = 0;
-    d0.x_len = 0;
-    d0.n_slash = 0;
-    ClassDyn& d1 = dyn(dp, c1.dyn);
-    d1.nrows = c1_tot;
-    d1.qrow0 = (c0_tot + TILE - 1) / TILE * TILE;
-    d1.x_len = g_tot;
-    d1.n_slash = 0;
+  if (blockIdx.x == GM_BLOCKS - 1) {
+    for (int i = tot[0] + threadIdx.x; i < c1.x_cap; i += blockDim.x) xg[i] = POS_PAD;
+    if (threadIdx.x == 0) {
+      ClassDyn& d0 = dyn(dp, c0.dyn);
+      d0.nrows = tot[1];
+      d0.qrow0 = 0;
+      d0.x_len = 0;
+      d0.n_slash = 0;
+      ClassDyn& d1 = dyn(dp, c1.dyn);
+      d1.nrows = tot[2];
+      d1.qrow0 = (tot[1] + TILE - 1) / TILE * TILE;
+      d1.x_len = tot[0];
+      d1.n_slash = 0;
+    }
   }
 }
 
@@ -725,10 +776,11 @@ cudaError_t launch_grid_detect(const DevPlan& dp, cudaStream_t st) {
 }
 
 cudaError_t launch_materialize(const DevPlan& dp, cudaStream_t st) {
-  count_launches(3);
+  count_launches(4);
   dyn_init_kernel<<<(dp.n_classes + 127) / 128, 128, 0, st>>>(dp);
   mat_lists_kernel<<<dp.n_classes, 512, 0, st>>>(dp);
-  grid_mat_kernel<<<dp.Hq, 1024, 0, st>>>(dp);
+  grid_count_kernel<<<dim3(GM_BLOCKS, dp.Hq), GM_THREADS, 0, st>>>(dp);
+  grid_write_kernel<<<dim3(GM_BLOCKS, dp.Hq), GM_THREADS, 0, st>>>(dp);
   for (int c = 0; c < dp.n_classes; ++c)
     if (dp.class_kind[c] == MSA_BLOCK) {
       count_launches(1);

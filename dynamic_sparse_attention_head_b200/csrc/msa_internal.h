@@ -95,7 +95,6 @@ struct HeadStatic {
   int64_t raws_off[2];       // int32 lists (offsets)
   int64_t counts_off;        // int32 [8]: n_v[0][0], n_v[0][1], n_v[1][0], n_v[1][1], n_s[0], n_s[1], stride, n_phases
   int64_t phases_off;        // int32 [max stride]
-  int64_t gmark_off;         // uint8 [L] grid marks
   int32_t blk_kmax, blk_nb;
   int32_t blk_fixed, _pad1;  // BLOCK: fixed top-k per row (> 0), else blk_budget
   double blk_budget;

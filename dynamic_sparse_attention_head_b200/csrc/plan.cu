@@ -572,7 +572,7 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
   for (int32_t h = 0; h < Hq; ++h) {
     HeadStatic& H = HS[h];
     const msa_head_cfg& cfg = P->heads[h];
-    H.counts_off = B.take(64);
+    H.counts_off = B.take(64 + 4 * 3 * 32);  // list counts; grid heads: per-block counts of the materialisation
     const bool per_seg = (cfg.flags & MSA_HEAD_PER_SEGMENT) != 0;  // lists live in the classes
     if ((cfg.kind == MSA_VSLASH || cfg.kind == MSA_QBOUND || cfg.kind == MSA_BOUND2D) && !per_seg) {
       for (int a = 0; a < 2; ++a) {
@@ -596,7 +596,6 @@ msa_status msa_plan_create(const msa_problem* prob, msa_plan** out) {
       int32_t smax = 1;
       for (int i = 0; i < cfg.n_strides; ++i) smax = std::max(smax, cfg.strides[i]);
       H.phases_off = B.take(4 * (int64_t)smax);
-      H.gmark_off = B.take(L);
     }
     if (cfg.kind == MSA_BLOCK) {
       int64_t kmax;
