@@ -609,10 +609,30 @@ __global__ void __launch_bounds__(TB_WARPS * 32) tiles_kernel(DevPlan dp, int bm
           for (int i = lane; i < nruns; i += 32)
             mark_units(bm, (int64_t)run_lo[i] - cs.band + 1, run_hi[i], kc_lo, hi_clip);
         if (cs.flags & CF_SLASH) {
+          // each lane takes a run of the (ascending) offsets; for one run of rows their key ranges
+          // descend, and two ranges less than a unit apart mark the same units as their hull (no
+          // unit fits in the gap), so the lane merges them and marks each merged range once
           const int32_t* sl = at<const int32_t>(dp, cs.slash_list_off);
-          for (int i = lane; i < cd.n_slash; i += 32) {
-            const int64_t o = sl[i];
-            for (int r = 0; r < nruns; ++r) mark_units(bm, run_lo[r] - o, run_hi[r] - o, kc_lo, hi_clip);
+          const int per = (cd.n_slash + 31) >> 5;
+          const int i0 = min(lane * per, cd.n_slash), i1 = min(i0 + per, cd.n_slash);
+          for (int r = 0; r < nruns; ++r) {
+            int64_t lo = 1, hi = 0;  // merged key range (empty)
+            for (int i = i0; i < i1; ++i) {
+              const int64_t o = sl[i];
+              int64_t a = run_lo[r] - o, b = run_hi[r] - o;  // clipped first: the gap rule holds inside
+              if (a < kc_lo) a = kc_lo;
+              if (b > hi_clip) b = hi_clip;
+              if (a > b) continue;
+              if (lo <= hi && b >= lo - UNIT && a <= hi + UNIT) {
+                lo = a < lo ? a : lo;
+                hi = b > hi ? b : hi;
+              } else {
+                if (lo <= hi) mark_units(bm, lo, hi, kc_lo, hi_clip);
+                lo = a;
+                hi = b;
+              }
+            }
+            if (lo <= hi) mark_units(bm, lo, hi, kc_lo, hi_clip);
           }
         }
         if (cs.flags & CF_BLOCK) {
