@@ -189,10 +189,20 @@ __global__ void grid_detect_kernel(DevPlan dp) {
       for (int g = 0; g < dp.n_segs; ++g) {
         if (seg[3 * g + 2] != MSA_VIDEO) continue;
         const int st = seg[3 * g], len = seg[3 * g + 1];
-        for (int t = p; t < len; t += s) {
-          if (have_v) sum += v[st + t];
-          ++cnt;
+        if (p >= len) continue;
+        cnt += (len - p + s - 1) / s;
+        if (!have_v) continue;
+        // four independent partial sums (loads in flight), combined in a fixed order
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        int t = p;
+        for (; t + 3 * s < len; t += 4 * s) {
+          a0 += v[st + t];
+          a1 += v[st + t + s];
+          a2 += v[st + t + 2 * s];
+          a3 += v[st + t + 3 * s];
         }
+        for (; t < len; t += s) a0 += v[st + t];
+        sum += (a0 + a1) + (a2 + a3);
       }
       const float mean = cnt > 0 ? sum / (float)cnt : 0.f;
       sc_cur[p] = mean;
@@ -791,7 +801,7 @@ cudaError_t launch_layout(const DevPlan& dp, cudaStream_t st) {
 
 cudaError_t launch_grid_detect(const DevPlan& dp, cudaStream_t st) {
   count_launches(1);
-  grid_detect_kernel<<<dp.Hq, 256, 0, st>>>(dp);
+  grid_detect_kernel<<<dp.Hq, 1024, 0, st>>>(dp);
   return cudaGetLastError();
 }
 
