@@ -255,7 +255,7 @@ msa_status msa_mask_pairs(const msa_plan* plan, void* ws, int64_t* counts, void*
 
 /* How msa_sparse_prefill divides its work (host only, no device access): out[0] = work units,
  * out[1] = key chunks, out[2] = unit bands (0 when the keys are not chunked).  When one head's
- * K and V exceed about 96 MB (L > 192K tokens) the keys are cut into chunks of 65536 (the
+ * K and V exceed about 96 MB (L > 192K tokens) the keys are cut into chunks of 131072 (the
  * environment variable MSA_ATTN_CHUNK_KEYS, a multiple of 128, read at msa_plan_create,
  * overrides the chunk size; 0 turns chunking off): the units of a band of work items then run
  * chunk by chunk so that the units in flight share one chunk of K and V in L2, and a work
