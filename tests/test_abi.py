@@ -84,6 +84,10 @@ def test_attention_units_chunking_rule(monkeypatch):
     assert msa.Plan(workload.qwen2_7b_video_128k()).attention_units()[1] == 1
     units, chunks = msa.Plan(workload.longvila_1m()).attention_units()
     assert chunks == 8
+    # the threshold: K and V of one head above 96 MB (L x 512 B), i.e. L > 196608
+    assert msa.Plan(workload.llama3_8b_text(L=196608)).attention_units()[1] == 1
+    assert msa.Plan(workload.llama3_8b_text(L=196672)).attention_units()[1] == 2
+    assert msa.Plan(workload.llama3_8b_text(L=262144)).attention_units()[1] == 2
     monkeypatch.setenv("MSA_ATTN_CHUNK_KEYS", "256")
     p = workload.llama3_8b_text(L=2048)
     assert msa.Plan(p).attention_units()[1] == 8
